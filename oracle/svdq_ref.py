@@ -1,0 +1,131 @@
+"""Reference (fp64, CPU) SVDQuant W4A4 NVFP4 linear layer.
+
+Test infrastructure only (see the package docstring).
+
+The layer, as the "nunchaku-z-image-turbo-svdq" model card writes it in
+"What's stored on disk":
+
+    y = scaled_mma(quant(x * smooth), qweight, ascales, wscales)
+        * wtscale * wcscales + (x @ proj_down) @ proj_up^T + bias
+
+with the operand table of the same section:
+
+    qweight   [N, K/2]  int8      FP4 nibble pack, low nibble = even k
+    wscales   [K/16, N] e4m3fn    one scale per 16 k per output channel
+    wcscales  [N]       bf16      per-output-channel scale
+    wtscale   [1]       bf16      global alpha
+    smooth    [K]       bf16      per-input-channel smoothing factor
+    proj_down [K, R]    bf16      SVD residual, down factor (R = 128)
+    proj_up   [N, R]    bf16      SVD residual, up factor
+
+Readings taken where the card is silent (each is listed in the design doc):
+
+* ``quant`` is dynamic NVFP4 quantization of each 16-element group along
+  K: scale = e4m3(amax / 6), element = E2M1(v / scale), both rounded to
+  nearest with ties to even and saturating; 6 is the largest E2M1
+  magnitude.  A group whose scale rounds to zero gets zero codes (sign
+  kept).
+* ``x * smooth`` is a multiply by the stored factor, computed exactly.
+* The low-rank branch takes the raw x, as the formula is written.
+* ``bias`` is an optional bf16 [N]; the card's table has no bias row.
+
+All arrays are NumPy; bf16 tensors are raw uint16 bit patterns and FP8 /
+FP4 tensors raw uint8 codes.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .nvfp4 import (
+    bf16_bits_to_f64,
+    decode_e2m1,
+    decode_e4m3,
+    encode_e2m1_rne_sat,
+    encode_e4m3_rne_satfinite,
+    pack_nibbles,
+    unpack_nibbles,
+)
+
+GROUP = 16          # elements per scale along K (model card, first paragraph)
+E2M1_MAX = 6.0      # largest E2M1 magnitude
+
+
+def quantize_act(x_bits, smooth_bits):
+    """quant(x * smooth) -> (qact [M, K/2] uint8, ascales [M, K/16] uint8).
+
+    Model card "What's stored on disk": the runtime formula's
+    ``quant(x * smooth)``, producing the same packed layout as qweight
+    (low nibble = even k) and one e4m3 scale per 16 k, as for wscales.
+
+    Steps, per row m and group g = k // 16:
+      1. v = x[m, k] * smooth[k] (exact in float64: both are bf16).
+      2. a = max_k |v| over the group.
+      3. s = e4m3_rne_satfinite(a / 6); d = decoded value of s.
+      4. code = E2M1_rne_sat(v / d), or a signed zero code if d == 0.
+      5. pack codes two per byte, low nibble = even k.
+    """
+    x = bf16_bits_to_f64(x_bits)
+    smooth = bf16_bits_to_f64(smooth_bits)
+    M, K = x.shape
+    assert K % GROUP == 0 and smooth.shape == (K,)
+    v = x * smooth[None, :]
+    vg = v.reshape(M, K // GROUP, GROUP)
+    amax = np.abs(vg).max(axis=2)
+    ascales = encode_e4m3_rne_satfinite(amax / E2M1_MAX)
+    d = decode_e4m3(ascales)[:, :, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(d == 0.0, 0.0 * vg, vg / np.where(d == 0.0, 1.0, d))
+    codes = encode_e2m1_rne_sat(q).reshape(M, K)
+    return pack_nibbles(codes), ascales
+
+
+def dequant_act(qact, ascales):
+    """Decoded activation operand [M, K] float64: e2m1(code) * e4m3(scale)."""
+    a = decode_e2m1(unpack_nibbles(qact))
+    s = decode_e4m3(ascales)
+    return a * np.repeat(s, GROUP, axis=1)
+
+
+def dequant_weight(qweight, wscales):
+    """Decoded weight [N, K] float64 from qweight [N, K/2], wscales [K/16, N]."""
+    w = decode_e2m1(unpack_nibbles(qweight))
+    s = decode_e4m3(wscales).T                     # -> [N, K/16]
+    return w * np.repeat(s, GROUP, axis=1)
+
+
+def lowrank_down(x_bits, proj_down_bits):
+    """L = x @ proj_down, float64 [M, R] (model card runtime formula)."""
+    return bf16_bits_to_f64(x_bits) @ bf16_bits_to_f64(proj_down_bits)
+
+
+def w4a4_linear(qact, ascales, qweight, wscales, wcscales_bits, wtscale_bits,
+                proj_up_bits, bias_bits, L):
+    """y = scaled_mma(...) * wtscale * wcscales + L @ proj_up^T + bias.
+
+    ``scaled_mma`` is the block-scaled product
+    acc[m, n] = sum_k e2m1(qa[m,k]) sa[m,k/16] e2m1(qw[n,k]) sw[k/16,n],
+    done as one float64 matmul of the decoded operands.  ``L`` is the
+    low-rank down product (float64 [M, R]); ``bias_bits`` may be None.
+    Returns float64 [M, N].
+    """
+    acc = dequant_act(qact, ascales) @ dequant_weight(qweight, wscales).T
+    alpha = bf16_bits_to_f64(np.asarray(wtscale_bits).reshape(-1))[0]
+    c = bf16_bits_to_f64(wcscales_bits)
+    y = acc * alpha * c[None, :] + L @ bf16_bits_to_f64(proj_up_bits).T
+    if bias_bits is not None:
+        y = y + bf16_bits_to_f64(bias_bits)[None, :]
+    return y
+
+
+def svdq_linear_from_x(x_bits, smooth_bits, proj_down_bits, qweight, wscales,
+                       wcscales_bits, wtscale_bits, proj_up_bits, bias_bits):
+    """The whole layer from raw x: quantize, low-rank down, then the linear.
+
+    Returns (y float64 [M, N], qact, ascales, L float64 [M, R]).
+    """
+    qact, ascales = quantize_act(x_bits, smooth_bits)
+    L = lowrank_down(x_bits, proj_down_bits)
+    y = w4a4_linear(qact, ascales, qweight, wscales, wcscales_bits,
+                    wtscale_bits, proj_up_bits, bias_bits, L)
+    return y, qact, ascales, L
