@@ -1,0 +1,453 @@
+"""Throughput of the SVDQuant W4A4 NVFP4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = the whole per-forward path on one batch of synthetic input:
+svdq_quantize_act (smooth + NVFP4 quantize + low-rank down) then
+svdq_w4a4_linear (block-scaled FP4 GEMM + fused epilogue).  The one-time
+svdq_repack_weights is timed separately (config.repack_us).
+
+Metric: TFLOP/s = (2 M N K + 2 M R (K + N)) / step time.  Default workload:
+the qkv projection of a 30-block DiT, M = 4352 tokens, K = 3840,
+N = 11520, R = 128.  Inputs rotate over several sets whose total exceeds
+the 126 MB L2, so every step reads weights and activations from HBM.
+
+Under torchrun each rank runs its own batch of the same shape (the layer
+is independent per token: weak scaling, no collective on the data path);
+the time is the max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SVDQ W4A4 linear TFLOP/s & % of dense NVFP4 roofline at DiT shapes"
+UNIT = "TFLOP/s"
+R = 128
+L2_BYTES = 126 * 1024 * 1024
+FP4_OVER_BF16 = 4.0   # nominal dense FP4 : BF16 tensor ratio (9 : 2.25 PFLOP/s)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qkv_m4352_k3840_n11520")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def flops_per_step(M, K, N):
+    return 2 * M * N * K + 2 * M * R * (K + N)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+def load_traffic(kernel_key):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if any."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        for line in open(path):
+            parts = line.split()
+            if len(parts) >= 2 and parts[0] == kernel_key:
+                return float(parts[1])
+    except OSError:
+        pass
+    return None
+
+
+# ------------------------------------------------------------ clocks ----
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 8:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for n, v in zip(names, s[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# -------------------------------------------------------- distributed ----
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------ our CUDA path ----
+
+def make_sets(M, K, N, nsets, seed, dev):
+    import torch
+    from nvfp4_w4a4_quantized_smooth_b200 import svdq, synth
+    sets = []
+    for i in range(nsets):
+        L = synth.make_layer(M, K, N, seed=seed + i)
+        d = {k: (None if v is None else v.to(dev)) for k, v in vars(L).items()}
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        d["wscales_tiled"] = svdq.repack_weights(d["wscales"])
+        d["repack_s"] = time.perf_counter() - t0
+        d["qact"] = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        d["asc"] = torch.empty(svdq.ascales_tiled_bytes(M, K), dtype=torch.uint8, device=dev)
+        d["lr"] = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
+        d["y"] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        sets.append(d)
+    return sets
+
+
+def set_bytes(d):
+    import torch
+    return sum(v.numel() * v.element_size() for v in d.values() if isinstance(v, torch.Tensor))
+
+
+def run_step(svdq, d, stream, ev=None):
+    if ev is not None:
+        ev[0].record(stream)
+    svdq.quantize_act(d["x"], d["smooth"], d["proj_down"], qact=d["qact"], ascales_tiled=d["asc"],
+                      lowrank=d["lr"], stream=stream)
+    if ev is not None:
+        ev[1].record(stream)
+    svdq.w4a4_linear(d["qact"], d["asc"], d["lr"], d["qweight"], d["wscales_tiled"],
+                     d["wcscales"], d["wtscale"], d["proj_up"], d["bias"], y=d["y"],
+                     stream=stream)
+    if ev is not None:
+        ev[2].record(stream)
+
+
+def bench_ours(args, world, rank, local):
+    import torch
+    from nvfp4_w4a4_quantized_smooth_b200 import build as b
+    if rank == 0:
+        b.build()
+    barrier(world)
+    from nvfp4_w4a4_quantized_smooth_b200 import svdq, synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    M, K, N = synth.WORKLOADS[args.workload]
+    seed = synth.workload_seed(args.workload) + 7919 * rank
+    one = flops_per_step(M, K, N)
+
+    # rotating sets: enough that a set is evicted from L2 before it returns
+    probe = make_sets(M, K, N, 1, seed, dev)
+    per_set = set_bytes(probe[0])
+    nsets = max(3, -(-3 * L2_BYTES // per_set))
+    sets = probe + make_sets(M, K, N, nsets - 1, seed + 1, dev)
+    repack_us = 1e6 * statistics.median(d["repack_s"] for d in sets)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            run_step(svdq, sets[i % nsets], stream)
+        svdq.check_device_error(stream)
+
+        K_steps = args.steps
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                              int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+        clocks.start()
+        time.sleep(0.2)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for i in range(K_steps):
+            run_step(svdq, sets[i % nsets], stream, evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        clocks.stop()
+        svdq.check_device_error(stream)
+
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
+    kq_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    kg_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    kq_avg = sum(kq_ms) / K_steps
+    kg_avg = sum(kg_ms) / K_steps
+
+    value = one * K_steps * world / (elapsed_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+
+    # roofline of the whole step and of each kernel
+    bytes_kq = 2 * M * K + 2 * K + 2 * K * R + M * K // 2 + M * K // 16 + 2 * M * R
+    bytes_kg = (M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + 4 * N + 2 + 2 * M * R
+                + 2 * N * R + 2 * M * N)
+    flops_kg = 2 * M * N * K + 2 * M * R * N
+    t_roof_step = max(one / (fp4_peak * 1e12), (bytes_kq + bytes_kg) / (hbm * 1e9))
+    step_s = elapsed_ms * 1e-3 / K_steps
+    kg_tflops = flops_kg / (kg_avg * 1e-3) / 1e12
+    kq_gbs = bytes_kq / (kq_avg * 1e-3) / 1e9
+    traffic = load_traffic("w4a4_linear_kernel")
+
+    # end to end through the public API with host buffers
+    e2e = bench_e2e(args, svdq, sets[0], dev, M, K, N, world)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": K_steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(elapsed_ms / K_steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3 block16, fp32 accumulate) + bf16 low-rank",
+        "data": "synthetic (seeded; random weights of the layer's shapes)",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "R": R,
+                   "parallelism": f"dp{world} (independent token batches per GPU)",
+                   "l2": f"inputs larger than L2: {nsets} rotating sets x "
+                         f"{per_set / 2**20:.0f} MiB",
+                   "repack_us": round(repack_us, 1),
+                   "roofline_frac_of_step": round(t_roof_step / step_s, 4)},
+        "roofline": {"bound": "tensor", "kernel": "w4a4_linear_kernel",
+                     "achieved": round(kg_tflops, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(kg_tflops / fp4_peak, 4),
+                     "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal "
+                                    "FP4:BF16 dense ratio)",
+                     "algorithmic_flops_per_launch": flops_kg,
+                     "avg_launch_ms": round(kg_avg, 5)},
+        "kernels": {
+            "quantize_act_kernel": {"avg_ms": round(kq_avg, 5), "bytes": bytes_kq,
+                                    "GB/s": round(kq_gbs, 1), "peak_GB/s": hbm,
+                                    "frac": round(kq_gbs / hbm, 4), "bound": "hbm"},
+            "w4a4_linear_kernel": {"avg_ms": round(kg_avg, 5), "flops": flops_kg,
+                                   "TFLOP/s": round(kg_tflops, 1), "bytes": bytes_kg},
+        },
+        "e2e": e2e,
+        "gpu_launches": 2 * K_steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, sample_rows=256)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def bench_e2e(args, svdq, d, dev, M, K, N, world):
+    """Same metric through the public API with the input in pinned host
+    memory and the output read back to pinned host memory every step."""
+    import torch
+    stream = torch.cuda.Stream(device=dev)
+    x_host = d["x"].cpu().pin_memory()
+    y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(d["x"])
+    steps = max(args.e2e_steps, 1)
+    with torch.cuda.stream(stream):
+        def one_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            svdq.quantize_act(x_dev, d["smooth"], d["proj_down"], qact=d["qact"],
+                              ascales_tiled=d["asc"], lowrank=d["lr"], stream=stream)
+            svdq.w4a4_linear(d["qact"], d["asc"], d["lr"], d["qweight"], d["wscales_tiled"],
+                             d["wcscales"], d["wtscale"], d["proj_up"], d["bias"], y=d["y"],
+                             stream=stream)
+            y_host.copy_(d["y"], non_blocking=True)
+        for _ in range(3):
+            one_step()
+        torch.cuda.synchronize(dev)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        s.record(stream)
+        for _ in range(steps):
+            one_step()
+        e.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    val = flops_per_step(M, K, N) * steps * world / (ms * 1e-3) / 1e12
+    return {"value": round(val, 2), "unit": UNIT,
+            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
+
+
+# ------------------------------------------------------- the oracle ------
+
+def cpu_baseline(workload, sample_rows=256, min_seconds=10.0):
+    """The fp64 CPU oracle, as it stands, on a bounded sample of the workload:
+    `sample_rows` tokens of the same layer (all K, all N), repeated until
+    `min_seconds` of CPU work.  Returns the metric in TFLOP/s."""
+    from nvfp4_w4a4_quantized_smooth_b200 import synth
+    from oracle import svdq_ref as ref
+    M, K, N = synth.WORKLOADS[workload]
+    rows = min(sample_rows, M)
+    L = synth.make_layer(rows, K, N, seed=synth.workload_seed(workload))
+    b = synth.bits
+    args = (b(L.x), b(L.smooth), b(L.proj_down), b(L.qweight), b(L.wscales), b(L.wcscales),
+            b(L.wtscale), b(L.proj_up), b(L.bias))
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        ref.svdq_linear_from_x(*args)
+        reps += 1
+        if time.perf_counter() - t0 >= min_seconds:
+            break
+    dt = time.perf_counter() - t0
+    value = flops_per_step(rows, K, N) * reps / dt / 1e12
+    return {"value": round(value, 6), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{rows} of {M} tokens of {workload} (all K, all N), {reps} passes, "
+                      f"{dt:.1f} s"}
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def bench_reference(args, world, rank):
+    """The oracle (CPU, fp64) as the reference arm, rank 0 only."""
+    if rank != 0:
+        return
+    from nvfp4_w4a4_quantized_smooth_b200 import synth
+    from oracle import svdq_ref as ref
+    M, K, N = synth.WORKLOADS[args.workload]
+    rows = min(32, M)
+    L = synth.make_layer(rows, K, N, seed=synth.workload_seed(args.workload))
+    b = synth.bits
+    a = (b(L.x), b(L.smooth), b(L.proj_down), b(L.qweight), b(L.wscales), b(L.wcscales),
+         b(L.wtscale), b(L.proj_up), b(L.bias))
+    for _ in range(min(args.warmup, 1)):
+        ref.svdq_linear_from_x(*a)
+    steps = max(1, min(args.steps, 20))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        ref.svdq_linear_from_x(*a)
+    dt = time.perf_counter() - t0
+    value = flops_per_step(rows, K, N) * steps / dt / 1e12
+    sample = f"each step: {rows} of {M} tokens of {args.workload} (all K, all N)"
+    out = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": min(args.warmup, 1), "ms_per_step": round(1e3 * dt / steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
+        "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "R": R},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _blas_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        bench_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        bench_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * svdq.h -- C ABI of libsvdq.so, the SVDQuant W4A4 NVFP4 linear layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (nunchaku-z-image-turbo-svdq model card, "What's stored on
+ * disk", runtime formula):
+ *
+ *   y = scaled_mma(quant(x * smooth), qweight, ascales, wscales)
+ *       * wtscale * wcscales + (x @ proj_down) @ proj_up^T + bias
+ *
+ * Operand layouts follow the same section's table: qweight [N, K/2] FP4
+ * E2M1 nibble pack with the low nibble holding the even k; wscales
+ * [K/16, N] float8_e4m3fn; wcscales [N], wtscale [1], smooth_factor [K]
+ * bf16; proj_down [K, R] and proj_up [N, R] bf16 with R = 128.  The NVFP4
+ * format (E2M1 elements, one e4m3 scale per 16 elements along K) is the
+ * one the card's first paragraph names; the E2M1 bit layout is the one the
+ * Z-Image NVFP4 blog gives in "NVFP4 技术背景".
+ *
+ * The path is three calls: svdq_repack_weights (once per layer),
+ * svdq_quantize_act and svdq_w4a4_linear (per forward).
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Types: bf16 tensors are passed as raw 16-bit patterns (uint16_t);
+ *   FP4 / FP8 tensors as raw bytes.  All matrices are row-major with the
+ *   last index contiguous.
+ * - Memory: every tensor pointer is a DEVICE pointer on the current CUDA
+ *   device, unless a parameter says otherwise.  The caller owns and
+ *   allocates every buffer (sizes from the svdq_*_bytes queries); the
+ *   library allocates nothing apart from a few static device words (an
+ *   error word and a counter).
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = the
+ *   legacy default stream).  Calls only enqueue work and return; nothing
+ *   synchronizes the host except where a call says so.
+ * - Alignment: tensor pointers must be 16-byte aligned (wtscale: 2 bytes).
+ * - Errors: arguments are checked before anything is enqueued; a failing
+ *   check returns its status and enqueues nothing.  A launch failure
+ *   returns SVDQ_ERR_CUDA.  Every wait inside the kernels is bounded;
+ *   a kernel that gives up records it in a device error word and returns,
+ *   and svdq_check_device_error reports it as SVDQ_ERR_TIMEOUT.  A
+ *   recorded error makes later kernels return early until it is read.
+ * - Device: the calls run only on compute capability 10.0 (B200, sm_100a);
+ *   anything else gives SVDQ_ERR_ARCH.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,  /* null pointer, bad scale byte, bad value   */
+  SVDQ_ERR_SHAPE = 2,        /* M, N < 1, K not a positive multiple of 16 */
+  SVDQ_ERR_ALIGNMENT = 3,    /* pointer or leading dimension misaligned   */
+  SVDQ_ERR_UNSUPPORTED = 4,  /* valid but not implemented (R, K, N limits)*/
+  SVDQ_ERR_ARCH = 5,         /* current device is not sm_100              */
+  SVDQ_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed      */
+  SVDQ_ERR_TIMEOUT = 7       /* a kernel's bounded wait ran out           */
+} svdq_status;
+
+/* Human-readable name of a status code.  Never NULL; static storage. */
+const char* svdq_status_string(int status);
+
+/* ABI version of this header (bumped on any signature change). */
+#define SVDQ_ABI_VERSION 1
+int svdq_abi_version(void);
+
+/* ---- size queries (bytes the caller allocates) ------------------------ */
+
+/* Tiled activation scales written by svdq_quantize_act for an [M, K]
+ * input: ceil(M/128) * (K/64) blocks of 512 bytes.  0 on bad arguments. */
+size_t svdq_ascales_tiled_bytes(int M, int K);
+
+/* Tiled weight scales written by svdq_repack_weights for N output
+ * channels: ceil(N/256)*2 * (K/64) blocks of 512 bytes.  0 on bad args. */
+size_t svdq_wscales_tiled_bytes(int N, int K);
+
+/* Low-rank activations L = x @ proj_down written by svdq_quantize_act:
+ * M * R bf16 values ([M, R] row-major). */
+size_t svdq_lowrank_bytes(int M, int R);
+
+/* ---- the path ---------------------------------------------------------- */
+
+/* One-time conversion of the on-disk weight scales into the tile order the
+ * GEMM reads (model card, "What's stored on disk": wscales [K/16, N]
+ * float8_e4m3fn; the card's "Why row-major" section allows a one-shot
+ * load-time pack).
+ *   wscales        [K/16, N] e4m3fn codes, device.
+ *   N, K           output channels, input channels (K % 64 == 0).
+ *   wscales_tiled  device, svdq_wscales_tiled_bytes(N, K) bytes; written
+ *                  completely (padding rows get scale 0).
+ * The GEMM reads scales as unsigned e4m3, so a byte with the sign bit set,
+ * or a NaN code (0x7F), is rejected: the call then returns
+ * SVDQ_ERR_INVALID_ARG.  To report that, this call SYNCHRONIZES `stream`. */
+int svdq_repack_weights(const uint8_t* wscales, int N, int K,
+                        void* wscales_tiled, void* stream);
+
+/* Activation side of the layer (model card runtime formula): reads x once
+ * and writes quant(x * smooth) and the low-rank product x @ proj_down.
+ *   x           [M, ldx] bf16, first K columns used; ldx >= K, ldx % 8 == 0.
+ *   smooth      [K] bf16 smoothing factor (multiplied, not divided).
+ *   proj_down   [K, R] bf16.
+ *   R           rank; only 128 is supported (else SVDQ_ERR_UNSUPPORTED).
+ *   qact        out, [M, K/2] bytes: E2M1 codes, low nibble = even k.
+ *   ascales_tiled out, svdq_ascales_tiled_bytes(M, K) bytes: one e4m3
+ *               scale per 16 k per row, scale = e4m3(amax/6), elements
+ *               E2M1(v/scale); both rounded to nearest-even, saturating.
+ *               Read its logical [M, K/16] form with svdq_unpack_scales.
+ *   lowrank     out, [M, R] bf16: x @ proj_down accumulated in fp32 and
+ *               rounded to bf16 (the raw x, not x * smooth).
+ * Limits: K % 64 == 0 (else SVDQ_ERR_UNSUPPORTED). */
+int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx,
+                      const uint16_t* smooth, const uint16_t* proj_down, int R,
+                      uint8_t* qact, void* ascales_tiled, uint16_t* lowrank,
+                      void* stream);
+
+/* Block-scaled FP4 GEMM with the fused epilogue (model card runtime
+ * formula):
+ *   y[m, n] = acc[m, n] * wtscale * wcscales[n]
+ *             + sum_r lowrank[m, r] * proj_up[n, r] + bias[n],
+ *   acc[m, n] = sum_k e2m1(qact[m,k]) * sa[m,k/16] * e2m1(qweight[n,k])
+ *                     * sw[k/16,n],
+ * accumulated in fp32 and stored as bf16 (nearest-even).
+ *   qact, ascales_tiled, lowrank  as written by svdq_quantize_act.
+ *   qweight        [N, K/2] bytes (on-disk layout).
+ *   wscales_tiled  as written by svdq_repack_weights.
+ *   wcscales [N], wtscale [1] (read on the device), proj_up [N, R],
+ *   bias [N] or NULL: bf16.
+ *   y              out, [M, ldy] bf16, ldy >= N, ldy % 8 == 0.
+ * Limits: R == 128, K % 256 == 0, N % 32 == 0 (else SVDQ_ERR_UNSUPPORTED). */
+int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
+                     const uint16_t* lowrank, const uint8_t* qweight,
+                     const void* wscales_tiled, const uint16_t* wcscales,
+                     const uint16_t* wtscale, const uint16_t* proj_up,
+                     const uint16_t* bias, int M, int N, int K, int R,
+                     uint16_t* y, int ldy, void* stream);
+
+/* ---- helpers ------------------------------------------------------------ */
+
+/* Inverse of the tile order, for tests and inspection: tiled scales of
+ * `rows` rows (M for activations, N for weights) -> out [rows, K/16]
+ * bytes, device.  For weights this is the transpose of the on-disk
+ * wscales [K/16, N]. */
+int svdq_unpack_scales(const void* scales_tiled, int rows, int K,
+                       uint8_t* out, void* stream);
+
+/* out[i] = silu(a[i]) * b[i] in fp32, rounded to bf16; n elements.  Used
+ * to form the w2 input of a DiT feed-forward block (w2(silu(w1 x) * w3 x)). */
+int svdq_silu_mul(const uint16_t* a, const uint16_t* b, uint16_t* out,
+                  size_t n, void* stream);
+
+/* Synchronizes `stream`, then reads and clears this device's error word.
+ * Returns SVDQ_OK, SVDQ_ERR_TIMEOUT (a bounded wait ran out) or
+ * SVDQ_ERR_CUDA (a sticky launch / runtime error). */
+int svdq_check_device_error(void* stream);
+
+/* Sets the limit of every bounded wait inside the kernels, in nanoseconds
+ * of GPU time, for the current device (default 2e9 = 2 s).  0 restores the
+ * default.  A short limit is how tests make a wait run out on purpose. */
+int svdq_set_wait_timeout_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

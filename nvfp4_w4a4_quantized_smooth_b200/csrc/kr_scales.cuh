@@ -1,0 +1,107 @@
+// kr_scales.cuh -- scale-factor tile order, and two small elementwise
+// kernels (scale unpack for tests, SiLU * mul for the feed-forward block).
+//
+// Tile order of every scale buffer the GEMM reads (activation scales and
+// weight scales alike): rows are cut into tiles of 128, K into blocks of
+// 64 (4 scales of 16).  Each (row tile t, K block b) pair is one 512-byte
+// block at offset (t * (K/64) + b) * 512, holding scale (row, 4 b + j) at
+// byte (row % 32) * 16 + ((row % 128) / 32) * 4 + j.  That is the layout
+// tcgen05.cp (32x128b, warpx4) turns into the TMEM scale-factor layout of
+// tcgen05.mma kind::mxf4nvf4: TMEM lane row % 32 (in every lane quarter),
+// column (row % 128) / 32, byte j.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace svdq {
+namespace kr {
+
+__device__ __forceinline__ size_t tiled_offset(int row, int kg, int kblocks) {
+  const int t = row >> 7, b = kg >> 2, j = kg & 3;
+  return (static_cast<size_t>(t) * kblocks + b) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + j;
+}
+
+// Device counter of rejected scale bytes (sign bit set, or NaN 0x7F).
+__device__ uint32_t g_bad_scales = 0;
+
+// wscales [K/16, N] (N contiguous) -> tiled, rows padded to `rows_pad`
+// with zero scales.  One thread per output word (4 scales of one row).
+__global__ void repack_weight_scales_kernel(const uint8_t* __restrict__ ws, int N, int K,
+                                            int rows_pad, uint8_t* __restrict__ out) {
+  const int kblocks = K / 64;
+  const size_t words = static_cast<size_t>(rows_pad) * kblocks;  // 4 bytes per (row, block)
+  uint32_t bad = 0;
+  for (size_t w = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; w < words;
+       w += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    // w enumerates the tiled buffer word by word: block index, then the
+    // word inside the 512-byte block.
+    const size_t blk = w >> 7;
+    const int wi = static_cast<int>(w & 127);
+    const int t = static_cast<int>(blk / kblocks);
+    const int b = static_cast<int>(blk % kblocks);
+    const int row = t * 128 + ((wi & 3) << 5) + (wi >> 2);
+    uint32_t word = 0;
+    if (row < N) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t v = ws[static_cast<size_t>(4 * b + j) * N + row];
+        if ((v & 0x80u) || v == 0x7Fu) ++bad;
+        word |= v << (8 * j);
+      }
+    }
+    reinterpret_cast<uint32_t*>(out)[w] = word;
+  }
+  if (bad) atomicAdd(&g_bad_scales, bad);
+}
+
+// tiled -> [rows, K/16] (row-major), the logical scale matrix.
+__global__ void unpack_scales_kernel(const uint8_t* __restrict__ tiled, int rows, int K,
+                                     uint8_t* __restrict__ out) {
+  const int kg_n = K / 16;
+  const size_t total = static_cast<size_t>(rows) * kg_n;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(i / kg_n);
+    const int kg = static_cast<int>(i % kg_n);
+    out[i] = tiled[tiled_offset(row, kg, K / 64)];
+  }
+}
+
+// out = silu(a) * b = a / (1 + exp(-a)) * b, fp32 math, bf16 result.
+__global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
+                                const __nv_bfloat16* __restrict__ b,
+                                __nv_bfloat16* __restrict__ out, size_t n) {
+  const size_t nvec = n / 8;
+  const uint4* a4 = reinterpret_cast<const uint4*>(a);
+  const uint4* b4 = reinterpret_cast<const uint4*>(b);
+  uint4* o4 = reinterpret_cast<uint4*>(out);
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < nvec;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 ua = __ldg(a4 + i), ub = __ldg(b4 + i);
+    const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
+    const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
+    uint32_t wo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a0 = __uint_as_float(wa[j] << 16), a1 = __uint_as_float(wa[j] & 0xFFFF0000u);
+      const float b0 = __uint_as_float(wb[j] << 16), b1 = __uint_as_float(wb[j] & 0xFFFF0000u);
+      const float o0 = a0 / (1.0f + expf(-a0)) * b0;
+      const float o1 = a1 / (1.0f + expf(-a1)) * b1;
+      __nv_bfloat162 r = __floats2bfloat162_rn(o0, o1);
+      wo[j] = *reinterpret_cast<uint32_t*>(&r);
+    }
+    o4[i] = make_uint4(wo[0], wo[1], wo[2], wo[3]);
+  }
+  // tail
+  const size_t tail0 = nvec * 8;
+  const size_t tid = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (tail0 + tid < n) {
+    const float av = __bfloat162float(a[tail0 + tid]);
+    const float bv = __bfloat162float(b[tail0 + tid]);
+    out[tail0 + tid] = __float2bfloat16_rn(av / (1.0f + expf(-av)) * bv);
+  }
+}
+
+}  // namespace kr
+}  // namespace svdq

@@ -1,0 +1,316 @@
+// svdq.cu -- the C ABI of libsvdq.so (declared in include/svdq.h):
+// argument checks, TMA descriptor encoding, launch configuration.  All
+// arithmetic of the layer happens in the kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "svdq.h"
+#include "sm100_ptx.cuh"
+#include "kq_quantize_act.cuh"
+#include "kg_w4a4_linear.cuh"
+#include "kr_scales.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool init = false;
+  bool sm100 = false;
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Per-device one-time set-up: architecture check, SM count, kernel
+// attributes.  Returns SVDQ_OK or an error status.
+int device_setup(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    d.sm100 = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    if (d.sm100) {
+      if (cudaFuncSetAttribute(svdq::kq::quantize_act_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               svdq::kq::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(svdq::kg::w4a4_linear_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               svdq::kg::SMEM_BYTES) != cudaSuccess)
+        return SVDQ_ERR_CUDA;
+    }
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return SVDQ_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.init = true;
+  }
+  if (!d.sm100) return SVDQ_ERR_ARCH;
+  *out = &d;
+  return SVDQ_OK;
+}
+
+// 2-D tensor map over a row-major matrix: `inner` contiguous elements per
+// row (row pitch `pitch_bytes`), `outer` rows; box `box_inner` x
+// `box_outer`, 128-byte swizzle, zero fill outside the matrix.
+int make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
+              uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+int grid_for(size_t work, int threads, int num_sms) {
+  size_t blocks = (work + threads - 1) / threads;
+  size_t cap = static_cast<size_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return static_cast<int>(blocks);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* svdq_status_string(int status) {
+  switch (status) {
+    case SVDQ_OK: return "SVDQ_OK";
+    case SVDQ_ERR_INVALID_ARG: return "SVDQ_ERR_INVALID_ARG: null pointer or invalid value";
+    case SVDQ_ERR_SHAPE: return "SVDQ_ERR_SHAPE: invalid M, N or K";
+    case SVDQ_ERR_ALIGNMENT: return "SVDQ_ERR_ALIGNMENT: pointer or leading dimension misaligned";
+    case SVDQ_ERR_UNSUPPORTED: return "SVDQ_ERR_UNSUPPORTED: shape outside the implemented limits";
+    case SVDQ_ERR_ARCH: return "SVDQ_ERR_ARCH: current device is not sm_100 (B200)";
+    case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA: CUDA runtime or launch error";
+    case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT: a bounded wait inside a kernel ran out";
+    default: return "SVDQ: unknown status";
+  }
+}
+
+int svdq_abi_version(void) { return SVDQ_ABI_VERSION; }
+
+size_t svdq_ascales_tiled_bytes(int M, int K) {
+  if (M < 1 || K < 64 || K % 64) return 0;
+  return static_cast<size_t>((M + 127) / 128) * (K / 64) * 512;
+}
+
+size_t svdq_wscales_tiled_bytes(int N, int K) {
+  if (N < 1 || K < 64 || K % 64) return 0;
+  return static_cast<size_t>((N + 255) / 256) * 2 * (K / 64) * 512;
+}
+
+size_t svdq_lowrank_bytes(int M, int R) {
+  if (M < 1 || R < 1) return 0;
+  return static_cast<size_t>(M) * R * 2;
+}
+
+int svdq_repack_weights(const uint8_t* wscales, int N, int K, void* wscales_tiled, void* stream) {
+  if (!wscales || !wscales_tiled) return SVDQ_ERR_INVALID_ARG;
+  if (N < 1 || K < 16 || K % 16) return SVDQ_ERR_SHAPE;
+  if (K % 64) return SVDQ_ERR_UNSUPPORTED;
+  if (!aligned(wscales_tiled, 16)) return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rows_pad = (N + 255) / 256 * 256;
+  const size_t words = static_cast<size_t>(rows_pad) * (K / 64);
+  uint32_t zero = 0, bad = 0;
+  if (cudaMemcpyToSymbolAsync(svdq::kr::g_bad_scales, &zero, sizeof(zero), 0,
+                              cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  svdq::kr::repack_weight_scales_kernel<<<grid_for(words, 256, d->num_sms), 256, 0, s>>>(
+      wscales, N, K, rows_pad, static_cast<uint8_t*>(wscales_tiled));
+  if (launch_status()) return SVDQ_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&bad, svdq::kr::g_bad_scales, sizeof(bad), 0,
+                                cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  return bad ? SVDQ_ERR_INVALID_ARG : SVDQ_OK;
+}
+
+int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* smooth,
+                      const uint16_t* proj_down, int R, uint8_t* qact, void* ascales_tiled,
+                      uint16_t* lowrank, void* stream) {
+  if (!x || !smooth || !proj_down || !qact || !ascales_tiled || !lowrank)
+    return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || K < 16 || K % 16 || ldx < K) return SVDQ_ERR_SHAPE;
+  if (R != svdq::kq::R || K % 64) return SVDQ_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(smooth, 16) || !aligned(proj_down, 16) || !aligned(qact, 16) ||
+      !aligned(ascales_tiled, 16) || !aligned(lowrank, 16) || ldx % 8)
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+
+  CUtensorMap tm_x, tm_pd;
+  if (make_tmap(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(ldx) * 2,
+                svdq::kq::BKE, svdq::kq::BM) ||
+      make_tmap(&tm_pd, proj_down, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, K,
+                static_cast<uint64_t>(R) * 2, 64, svdq::kq::BKE))
+    return SVDQ_ERR_CUDA;
+
+  const int m_tiles = (M + svdq::kq::BM - 1) / svdq::kq::BM;
+  const int chunks = K / svdq::kq::BKE;
+  // Split K over a cluster until the grid covers the SMs once.
+  int split = 1;
+  while (split < 8 && m_tiles * split * 2 <= d->num_sms && chunks >= split * 2) split *= 2;
+
+  svdq::kq::Params p;
+  p.smooth = reinterpret_cast<const __nv_bfloat16*>(smooth);
+  p.qact = qact;
+  p.ascales_tiled = static_cast<uint8_t*>(ascales_tiled);
+  p.lowrank = reinterpret_cast<__nv_bfloat16*>(lowrank);
+  p.M = M;
+  p.K = K;
+  p.chunks = chunks;
+  p.split = split;
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(split, m_tiles, 1);
+  cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = svdq::kq::SMEM_BYTES;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, svdq::kq::quantize_act_kernel, tm_x, tm_pd, p) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  return launch_status();
+}
+
+int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint16_t* lowrank,
+                     const uint8_t* qweight, const void* wscales_tiled, const uint16_t* wcscales,
+                     const uint16_t* wtscale, const uint16_t* proj_up, const uint16_t* bias, int M,
+                     int N, int K, int R, uint16_t* y, int ldy, void* stream) {
+  if (!qact || !ascales_tiled || !lowrank || !qweight || !wscales_tiled || !wcscales || !wtscale ||
+      !proj_up || !y)
+    return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 16 || K % 16 || ldy < N) return SVDQ_ERR_SHAPE;
+  if (R != 128 || K % svdq::kg::BK || N % 32) return SVDQ_ERR_UNSUPPORTED;
+  if (!aligned(qact, 16) || !aligned(ascales_tiled, 16) || !aligned(lowrank, 16) ||
+      !aligned(qweight, 16) || !aligned(wscales_tiled, 16) || !aligned(wcscales, 16) ||
+      !aligned(wtscale, 2) || !aligned(proj_up, 16) || (bias && !aligned(bias, 16)) ||
+      !aligned(y, 16) || ldy % 8)
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+
+  CUtensorMap tm_a, tm_b, tm_l, tm_p;
+  const uint64_t kb = static_cast<uint64_t>(K) / 2;
+  if (make_tmap(&tm_a, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, svdq::kg::BK_BYTES,
+                svdq::kg::BM) ||
+      make_tmap(&tm_b, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, N, kb, svdq::kg::BK_BYTES,
+                svdq::kg::BN) ||
+      make_tmap(&tm_l, lowrank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, M,
+                static_cast<uint64_t>(R) * 2, 64, svdq::kg::BM) ||
+      make_tmap(&tm_p, proj_up, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, N,
+                static_cast<uint64_t>(R) * 2, 64, svdq::kg::BN))
+    return SVDQ_ERR_CUDA;
+
+  svdq::kg::Params p;
+  p.ascales_tiled = static_cast<const uint8_t*>(ascales_tiled);
+  p.wscales_tiled = static_cast<const uint8_t*>(wscales_tiled);
+  p.wcscales = reinterpret_cast<const __nv_bfloat16*>(wcscales);
+  p.wtscale = reinterpret_cast<const __nv_bfloat16*>(wtscale);
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ldy = ldy;
+  p.m_tiles = (M + svdq::kg::BM - 1) / svdq::kg::BM;
+  p.n_tiles = (N + svdq::kg::BN - 1) / svdq::kg::BN;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = tiles < d->num_sms ? tiles : d->num_sms;
+  svdq::kg::w4a4_linear_kernel<<<grid, svdq::kg::NUM_THREADS, svdq::kg::SMEM_BYTES,
+                                 static_cast<cudaStream_t>(stream)>>>(tm_a, tm_b, tm_l, tm_p, p);
+  return launch_status();
+}
+
+int svdq_unpack_scales(const void* scales_tiled, int rows, int K, uint8_t* out, void* stream) {
+  if (!scales_tiled || !out) return SVDQ_ERR_INVALID_ARG;
+  if (rows < 1 || K < 16 || K % 16) return SVDQ_ERR_SHAPE;
+  if (K % 64) return SVDQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  const size_t total = static_cast<size_t>(rows) * (K / 16);
+  svdq::kr::unpack_scales_kernel<<<grid_for(total, 256, d->num_sms), 256, 0,
+                                   static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(scales_tiled), rows, K, out);
+  return launch_status();
+}
+
+int svdq_silu_mul(const uint16_t* a, const uint16_t* b, uint16_t* out, size_t n, void* stream) {
+  if (!a || !b || !out) return SVDQ_ERR_INVALID_ARG;
+  if (n == 0) return SVDQ_OK;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16)) return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  const size_t work = n / 8 > 8 ? n / 8 : 8;
+  svdq::kr::silu_mul_kernel<<<grid_for(work, 256, d->num_sms), 256, 0,
+                              static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(a), reinterpret_cast<const __nv_bfloat16*>(b),
+      reinterpret_cast<__nv_bfloat16*>(out), n);
+  return launch_status();
+}
+
+int svdq_check_device_error(void* stream) {
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  uint32_t w = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&w, svdq::g_error_word, sizeof(w)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (w) {
+    if (cudaMemcpyToSymbol(svdq::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+    return SVDQ_ERR_TIMEOUT;
+  }
+  return launch_status();
+}
+
+int svdq_set_wait_timeout_ns(uint64_t ns) {
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  const uint64_t v = ns ? ns : 2000000000ull;
+  if (cudaMemcpyToSymbol(svdq::g_wait_limit_ns, &v, sizeof(v)) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  return SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,231 @@
+"""Thin ctypes binding of libsvdq.so (include/svdq.h), same call names.
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  Tensors are torch CUDA tensors (torch supplies device
+memory and streams); each wrapper checks dtypes / contiguity, passes raw
+device pointers and the current stream, and raises ``SvdqError`` on a
+non-OK status.  There is no CPU fallback: if the library cannot be loaded
+the import of this module fails.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq.so")
+
+SVDQ_OK = 0
+SVDQ_ERR_INVALID_ARG = 1
+SVDQ_ERR_SHAPE = 2
+SVDQ_ERR_ALIGNMENT = 3
+SVDQ_ERR_UNSUPPORTED = 4
+SVDQ_ERR_ARCH = 5
+SVDQ_ERR_CUDA = 6
+SVDQ_ERR_TIMEOUT = 7
+
+# Every symbol include/svdq.h declares, with (restype, argtypes).
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "svdq_status_string": (ctypes.c_char_p, [_I]),
+    "svdq_abi_version": (_I, []),
+    "svdq_ascales_tiled_bytes": (_SZ, [_I, _I]),
+    "svdq_wscales_tiled_bytes": (_SZ, [_I, _I]),
+    "svdq_lowrank_bytes": (_SZ, [_I, _I]),
+    "svdq_repack_weights": (_I, [_P, _I, _I, _P, _P]),
+    "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
+    "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
+    "svdq_unpack_scales": (_I, [_P, _I, _I, _P, _P]),
+    "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
+    "svdq_check_device_error": (_I, [_P]),
+    "svdq_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
+}
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with "
+            "`python -m nvfp4_w4a4_quantized_smooth_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = load_library()
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.svdq_status_string(status).decode()
+        super().__init__(f"{where}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != SVDQ_OK:
+        raise SvdqError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str, dim: Optional[int] = None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dims")
+
+
+def abi_version() -> int:
+    return _lib.svdq_abi_version()
+
+
+def ascales_tiled_bytes(M: int, K: int) -> int:
+    return _lib.svdq_ascales_tiled_bytes(M, K)
+
+
+def wscales_tiled_bytes(N: int, K: int) -> int:
+    return _lib.svdq_wscales_tiled_bytes(N, K)
+
+
+def lowrank_bytes(M: int, R: int) -> int:
+    return _lib.svdq_lowrank_bytes(M, R)
+
+
+def repack_weights(wscales: torch.Tensor, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """wscales [K/16, N] uint8 (e4m3 codes) -> tiled scale buffer (uint8)."""
+    _need(wscales, torch.uint8, "wscales", 2)
+    wscales = wscales.contiguous()
+    K = wscales.shape[0] * 16
+    N = wscales.shape[1]
+    nbytes = wscales_tiled_bytes(N, K)
+    if out is None:
+        out = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=wscales.device)
+    _check(_lib.svdq_repack_weights(_ptr(wscales), N, K, _ptr(out), _stream(stream)),
+           "svdq_repack_weights")
+    return out
+
+
+def quantize_act(x: torch.Tensor, smooth: torch.Tensor, proj_down: torch.Tensor,
+                 qact: Optional[torch.Tensor] = None,
+                 ascales_tiled: Optional[torch.Tensor] = None,
+                 lowrank: Optional[torch.Tensor] = None, stream=None):
+    """x [M, K] bf16 (row stride may exceed K) -> (qact, ascales_tiled, lowrank)."""
+    _need(x, torch.bfloat16, "x", 2)
+    _need(smooth, torch.bfloat16, "smooth", 1)
+    _need(proj_down, torch.bfloat16, "proj_down", 2)
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along K")
+    M, K = x.shape
+    R = proj_down.shape[1]
+    dev = x.device
+    if qact is None:
+        qact = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    if ascales_tiled is None:
+        ascales_tiled = torch.empty(max(ascales_tiled_bytes(M, K), 1), dtype=torch.uint8,
+                                    device=dev)
+    if lowrank is None:
+        lowrank = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
+    _check(_lib.svdq_quantize_act(_ptr(x), M, K, x.stride(0), _ptr(smooth.contiguous()),
+                                  _ptr(proj_down.contiguous()), R, _ptr(qact),
+                                  _ptr(ascales_tiled), _ptr(lowrank), _stream(stream)),
+           "svdq_quantize_act")
+    return qact, ascales_tiled, lowrank
+
+
+def w4a4_linear(qact: torch.Tensor, ascales_tiled: torch.Tensor, lowrank: torch.Tensor,
+                qweight: torch.Tensor, wscales_tiled: torch.Tensor, wcscales: torch.Tensor,
+                wtscale: torch.Tensor, proj_up: torch.Tensor, bias: Optional[torch.Tensor],
+                y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The block-scaled FP4 GEMM with the fused epilogue -> y [M, N] bf16."""
+    _need(qact, torch.uint8, "qact", 2)
+    _need(qweight, torch.uint8, "qweight", 2)
+    _need(lowrank, torch.bfloat16, "lowrank", 2)
+    _need(proj_up, torch.bfloat16, "proj_up", 2)
+    M = qact.shape[0]
+    K = qact.shape[1] * 2
+    N = qweight.shape[0]
+    R = proj_up.shape[1]
+    if y is None:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=qact.device)
+    _check(_lib.svdq_w4a4_linear(_ptr(qact), _ptr(ascales_tiled), _ptr(lowrank),
+                                 _ptr(qweight), _ptr(wscales_tiled), _ptr(wcscales),
+                                 _ptr(wtscale), _ptr(proj_up), _ptr(bias), M, N, K, R,
+                                 _ptr(y), y.stride(0), _stream(stream)),
+           "svdq_w4a4_linear")
+    return y
+
+
+def unpack_scales(scales_tiled: torch.Tensor, rows: int, K: int, stream=None) -> torch.Tensor:
+    """Tiled scales -> logical [rows, K/16] uint8 (test / inspection helper)."""
+    out = torch.empty(rows, K // 16, dtype=torch.uint8, device=scales_tiled.device)
+    _check(_lib.svdq_unpack_scales(_ptr(scales_tiled), rows, K, _ptr(out), _stream(stream)),
+           "svdq_unpack_scales")
+    return out
+
+
+def silu_mul(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """silu(a) * b elementwise, bf16 (the w2 input of a DiT FFN block)."""
+    _need(a, torch.bfloat16, "a")
+    _need(b, torch.bfloat16, "b")
+    if a.shape != b.shape or not a.is_contiguous() or not b.is_contiguous():
+        raise ValueError("a and b must be contiguous with the same shape")
+    if out is None:
+        out = torch.empty_like(a)
+    _check(_lib.svdq_silu_mul(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream(stream)),
+           "svdq_silu_mul")
+    return out
+
+
+def check_device_error(stream=None) -> None:
+    """Synchronize the stream and raise if a kernel recorded an error."""
+    _check(_lib.svdq_check_device_error(_stream(stream)), "svdq_check_device_error")
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    _check(_lib.svdq_set_wait_timeout_ns(ns), "svdq_set_wait_timeout_ns")
+
+
+class PreparedWeights:
+    """One layer's device weights with the scales already repacked."""
+
+    def __init__(self, qweight, wscales, wcscales, wtscale, smooth, proj_down, proj_up,
+                 bias=None, stream=None):
+        self.qweight = qweight
+        self.wscales_tiled = repack_weights(wscales, stream=stream)
+        self.wcscales = wcscales
+        self.wtscale = wtscale
+        self.smooth = smooth
+        self.proj_down = proj_down
+        self.proj_up = proj_up
+        self.bias = bias
+        self.N = qweight.shape[0]
+        self.K = qweight.shape[1] * 2
+
+
+def svdq_linear(x: torch.Tensor, w: PreparedWeights, y: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Whole layer on device tensors: svdq_quantize_act then svdq_w4a4_linear."""
+    qact, asc, lr = quantize_act(x, w.smooth, w.proj_down, stream=stream)
+    return w4a4_linear(qact, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
+                       w.proj_up, w.bias, y=y, stream=stream)

@@ -1,0 +1,318 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Bit-exact: packed E2M1 codes, e4m3 activation scales, the repacked weight
+scales (round trip).  Within the stated tolerance: y and L.  All inputs are
+seeded synthetic operands of the shapes the layer runs at.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import nvfp4 as nv
+from oracle import svdq_ref as ref
+from nvfp4_w4a4_quantized_smooth_b200 import synth
+
+import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from nvfp4_w4a4_quantized_smooth_b200 import build
+    build.build()
+    torch.cuda.init()
+    yield
+
+
+# ------------------------------------------------------------- repack ---
+
+@pytest.mark.parametrize("N,K", [(512, 512), (96, 64), (100, 128), (3840, 3840), (11520, 3840),
+                                 (3840, 10240)])
+def test_repack_round_trip(N, K):
+    s = H.svdq()
+    g = torch.Generator().manual_seed(N + K)
+    ws = torch.randint(0, 0x7F, (K // 16, N), generator=g, dtype=torch.uint8)
+    t = s.repack_weights(ws.cuda())
+    assert t.numel() == s.wscales_tiled_bytes(N, K)
+    back = s.unpack_scales(t, N, K).cpu()
+    assert torch.equal(back, ws.t().contiguous())
+    # padding rows (beyond N) of the tiled buffer are zero scales
+    rows_pad = (N + 255) // 256 * 256
+    if rows_pad > N:
+        full = s.unpack_scales(t, rows_pad, K).cpu()
+        assert torch.all(full[N:] == 0)
+
+
+@pytest.mark.parametrize("bad", [0x80, 0xB8, 0x7F, 0xFF])
+def test_repack_rejects_sign_and_nan_scales(bad):
+    s = H.svdq()
+    ws = torch.full((8, 64), 0x38, dtype=torch.uint8)
+    ws[3, 17] = bad
+    with pytest.raises(s.SvdqError) as e:
+        s.repack_weights(ws.cuda())
+    assert e.value.status == s.SVDQ_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------- quantize ---
+
+@pytest.mark.parametrize("M,K", [(1, 64), (17, 128), (128, 512), (129, 512), (300, 192),
+                                 (64, 3840), (513, 1024), (16, 10240)])
+def test_quantize_act_bit_exact_and_lowrank(M, K):
+    s = H.svdq()
+    L = synth.make_layer(M, K, 32, seed=M * 7 + K)
+    qact, asc, lr = s.quantize_act(L.x.cuda(), L.smooth.cuda(), L.proj_down.cuda())
+    s.check_device_error()
+    q_ref, a_ref = H.oracle_quant(L.x, L.smooth)
+    H.assert_quant_exact(qact.cpu(), s.unpack_scales(asc, M, K).cpu(), q_ref, a_ref,
+                         f"M={M} K={K}")
+    L_ref = ref.lowrank_down(H.bits(L.x), H.bits(L.proj_down))
+    H.assert_lowrank_close(lr.cpu(), L_ref, f"M={M} K={K}")
+
+
+def _golden_rows():
+    """x rows built from the hand-worked groups of tests/golden/ (smooth = 1)."""
+    import test_oracle_pins as P
+    rows, scales, codes = [], [], []
+    for name in ("nvfp4_block_a.txt", "nvfp4_block_b.txt"):
+        g = P.read_golden(name)
+        rows.append([float(v) for v in g["v"]])
+        scales.append(int(g["scale"][0], 16))
+        codes.append([int(c, 16) for c in g["codes"]])
+    g = P.read_golden("nvfp4_block_c.txt")
+    for c in ("c1", "c2", "c3", "c4", "c5", "c6"):
+        rows.append([float(v) for v in g[c + "_v"]])
+        scales.append(int(g[c + "_scale"][0], 16))
+        codes.append([int(v, 16) for v in g[c + "_codes"]])
+    return rows, scales, codes
+
+
+def test_quantize_golden_groups_bit_exact():
+    # Each golden group is placed in every one of the 4 group slots of a
+    # 64-wide row (the other slots hold a plain group), so every position of
+    # the shared-memory swizzle and of the scale tile is exercised.
+    s = H.svdq()
+    rows, scales, codes = _golden_rows()
+    filler = [1.0] * 16
+    X, want_sc, want_codes = [], [], []
+    for gv, gs, gc in zip(rows, scales, codes):
+        for slot in range(4):
+            line = [filler] * 4
+            line[slot] = gv
+            X.append(sum(line, []))
+            want_sc.append((slot, gs))
+            want_codes.append((slot, gc))
+    M = len(X)
+    K = 64
+    x = torch.tensor(X, dtype=torch.float64).to(torch.bfloat16)
+    assert torch.equal(x.to(torch.float64), torch.tensor(X, dtype=torch.float64))
+    smooth = torch.ones(K, dtype=torch.bfloat16)
+    pd = torch.zeros(K, 128, dtype=torch.bfloat16)
+    qact, asc, lr = s.quantize_act(x.cuda(), smooth.cuda(), pd.cuda())
+    s.check_device_error()
+    asc_l = s.unpack_scales(asc, M, K).cpu().numpy()
+    cod = nv.unpack_nibbles(qact.cpu().numpy())
+    for m in range(M):
+        slot, gs = want_sc[m]
+        assert asc_l[m, slot] == gs, (m, hex(asc_l[m, slot]), hex(gs))
+        assert list(cod[m, 16 * slot:16 * slot + 16]) == want_codes[m][1], m
+    # and the oracle agrees everywhere (filler groups included)
+    q_ref, a_ref = H.oracle_quant(x, smooth)
+    H.assert_quant_exact(qact.cpu(), torch.from_numpy(asc_l), q_ref, a_ref, "golden rows")
+    assert torch.all(lr.cpu() == 0)
+
+
+def test_quantize_ties_signed_zeros_and_saturation():
+    # Elements planted on every E2M1 midpoint for many scales, signed zeros,
+    # tiny negatives, scale saturation and subnormal scales.
+    rng = np.random.default_rng(11)
+    rows = []
+    for scale_code in list(range(0x01, 0x7E, 3)):
+        d = float(nv.decode_e4m3(scale_code))
+        mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+        v = [6 * d] + [m * d for m in mids] + [-m * d for m in mids] + [-0.0]
+        rows.append(v)
+    rows.append([3e4, -2e4] + [0.0] * 14)
+    rows.append([-1e-3, 2e-3, -0.0, 0.0] * 4)
+    x = torch.tensor(rows, dtype=torch.float64).to(torch.bfloat16)
+    M = x.shape[0]
+    x = torch.cat([x, x.flip(1), x * 0.5, -x], dim=1)   # K = 64
+    smooth = torch.ones(64, dtype=torch.bfloat16)
+    s = H.svdq()
+    qact, asc, _ = s.quantize_act(x.cuda(), smooth.cuda(), torch.zeros(64, 128, dtype=torch.bfloat16).cuda())
+    s.check_device_error()
+    q_ref, a_ref = H.oracle_quant(x, smooth)
+    H.assert_quant_exact(qact.cpu(), s.unpack_scales(asc, M, 64).cpu(), q_ref, a_ref, "ties")
+
+
+def test_quantize_respects_row_stride():
+    s = H.svdq()
+    L = synth.make_layer(40, 256, 32, seed=5)
+    big = torch.zeros(40, 320, dtype=torch.bfloat16)
+    big[:, :256] = L.x
+    xd = big.cuda()[:, :256]
+    qact, asc, lr = s.quantize_act(xd, L.smooth.cuda(), L.proj_down.cuda())
+    s.check_device_error()
+    q_ref, a_ref = H.oracle_quant(L.x, L.smooth)
+    H.assert_quant_exact(qact.cpu(), s.unpack_scales(asc, 40, 256).cpu(), q_ref, a_ref, "stride")
+
+
+# ------------------------------------------------------------- linear ---
+
+@pytest.mark.parametrize("M,K,N", [(128, 512, 512), (1, 256, 256), (17, 256, 96), (200, 768, 288),
+                                   (129, 512, 544), (256, 1024, 768)])
+def test_linear_parity(M, K, N):
+    L = synth.make_layer(M, K, N, seed=M + 3 * K + 7 * N)
+    r = H.gpu_layer(L)
+    y_ref, q_ref, a_ref, _ = H.oracle_y(L)
+    H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, "quant")
+    H.assert_y_close(r["y"], y_ref, f"M={M} K={K} N={N}")
+
+
+def test_linear_without_bias():
+    L = synth.make_layer(64, 512, 256, seed=21, with_bias=False)
+    r = H.gpu_layer(L)
+    y_ref, *_ = H.oracle_y(L)
+    H.assert_y_close(r["y"], y_ref, "no bias")
+
+
+def test_integer_grid_invariant_bit_exact():
+    # Unit scales, no low-rank term, x groups on the E2M1 grid with amax 6:
+    # y must equal the bf16 rounding of the exact integer-grid product.
+    rng = np.random.default_rng(12)
+    M, K, N = 160, 512, 256
+    cx = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    cx[:, ::16] = 7
+    x = torch.from_numpy(nv.decode_e2m1(cx)).to(torch.bfloat16)
+    L = synth.make_layer(M, K, N, seed=13)
+    L.x = x
+    L.smooth = torch.ones(K, dtype=torch.bfloat16)
+    L.wscales = torch.full((K // 16, N), 0x38, dtype=torch.uint8)
+    L.wcscales = torch.ones(N, dtype=torch.bfloat16)
+    L.wtscale = torch.ones(1, dtype=torch.bfloat16)
+    L.proj_down = torch.zeros(K, 128, dtype=torch.bfloat16)
+    L.proj_up = torch.zeros(N, 128, dtype=torch.bfloat16)
+    L.bias = torch.zeros(N, dtype=torch.bfloat16)
+    r = H.gpu_layer(L)
+    y_ref, *_ = H.oracle_y(L)
+    want = nv.f64_to_bf16_bits_rne(y_ref)
+    got = H.bits(r["y"])
+    assert np.array_equal(got, want), f"{(got != want).sum()} outputs differ"
+
+
+def test_unit_scales_random_codes_exact():
+    # Same as above but with random per-block weight scales and wcscales that
+    # are powers of two: every product and partial sum stays exact in fp32.
+    rng = np.random.default_rng(14)
+    M, K, N = 128, 256, 256
+    cx = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    cx[:, ::16] = 7
+    x = torch.from_numpy(nv.decode_e2m1(cx)).to(torch.bfloat16)
+    L = synth.make_layer(M, K, N, seed=15)
+    L.x = x
+    L.smooth = torch.ones(K, dtype=torch.bfloat16)
+    L.wscales = torch.from_numpy(rng.choice([0x30, 0x38, 0x40, 0x48], (K // 16, N)).astype(np.uint8))
+    L.wcscales = torch.from_numpy(rng.choice([0.5, 1.0, 2.0], N)).to(torch.bfloat16)
+    L.wtscale = torch.ones(1, dtype=torch.bfloat16)
+    L.proj_down = torch.zeros(K, 128, dtype=torch.bfloat16)
+    L.proj_up = torch.zeros(N, 128, dtype=torch.bfloat16)
+    L.bias = torch.zeros(N, dtype=torch.bfloat16)
+    r = H.gpu_layer(L)
+    y_ref, *_ = H.oracle_y(L)
+    want = nv.f64_to_bf16_bits_rne(y_ref)
+    got = H.bits(r["y"])
+    assert np.array_equal(got, want), f"{(got != want).sum()} outputs differ"
+
+
+def test_zero_weights_give_lowrank_branch_only():
+    L = synth.make_layer(192, 512, 512, seed=16)
+    L.qweight = torch.zeros_like(L.qweight)
+    r = H.gpu_layer(L)
+    lr = (oracle.bf16_bits_to_f64(H.bits(L.x)) @ oracle.bf16_bits_to_f64(H.bits(L.proj_down))
+          @ oracle.bf16_bits_to_f64(H.bits(L.proj_up)).T
+          + oracle.bf16_bits_to_f64(H.bits(L.bias)))
+    H.assert_y_close(r["y"], lr, "low-rank only")
+
+
+def test_output_row_stride():
+    s = H.svdq()
+    L = synth.make_layer(100, 256, 256, seed=17)
+    d = H.to_dev(L)
+    wt = s.repack_weights(d["wscales"])
+    qact, asc, lr = s.quantize_act(d["x"], d["smooth"], d["proj_down"])
+    ybig = torch.full((100, 320), 7.0, dtype=torch.bfloat16, device="cuda")
+    s.w4a4_linear(qact, asc, lr, d["qweight"], wt, d["wcscales"], d["wtscale"], d["proj_up"],
+                  d["bias"], y=ybig[:, :256])
+    s.check_device_error()
+    y_ref, *_ = H.oracle_y(L)
+    H.assert_y_close(ybig[:, :256].cpu(), y_ref, "ldy")
+    assert torch.all(ybig[:, 256:].cpu() == 7.0)
+
+
+# ------------------------------------------------- full-size workloads ---
+
+def _full_size_check(name, n_rows=48):
+    M, K, N = synth.WORKLOADS[name]
+    L = synth.make_layer(M, K, N, seed=synth.workload_seed(name))
+    r = H.gpu_layer(L)
+    if M * K <= 20_000_000:
+        # every code and scale of the whole activation
+        q_ref, a_ref = H.oracle_quant(L.x, L.smooth)
+        H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, name)
+    rows = H.sample_rows(M, n_rows, seed=M)
+    y_ref, q_ref, a_ref, L_ref = H.oracle_y(L, rows=rows)
+    H.assert_quant_exact(r["qact"][rows], r["ascales"][rows], q_ref, a_ref, name)
+    H.assert_y_close(r["y"][rows], y_ref, name)
+    H.assert_lowrank_close(r["lowrank"][rows], L_ref, name)
+    return L, r
+
+
+def test_full_size_layer_m128():
+    _full_size_check("layer_m128_k512_n512", n_rows=128)
+
+
+def test_full_size_qkv():
+    _full_size_check("qkv_m4352_k3840_n11520")
+
+
+@pytest.mark.parametrize("M", synth.OUT_PROJ_SWEEP_M)
+def test_full_size_out_proj_sweep(M):
+    _full_size_check(f"out_m{M}_k3840_n3840", n_rows=32)
+
+
+def test_full_size_ffn_chain():
+    # w1, w3 on the block input, h = silu(y1) * y3 from the GPU's own bf16
+    # outputs, then w2 on h; the oracle for w2 takes that h as its input.
+    s = H.svdq()
+    L1, r1 = _full_size_check("ffn_w1_m4352_k3840_n10240", n_rows=24)
+    L3 = synth.make_layer(*synth.WORKLOADS["ffn_w3_m4352_k3840_n10240"],
+                          seed=synth.workload_seed("ffn_w3_m4352_k3840_n10240"))
+    L3.x = L1.x
+    r3 = H.gpu_layer(L3)
+    h = s.silu_mul(r1["y"].cuda(), r3["y"].cuda())
+    s.check_device_error()
+    a = r1["y"].float()
+    want_h = (a * torch.sigmoid(a) * r3["y"].float()).to(torch.bfloat16)
+    hd = h.cpu()
+    diff = (hd.float() - want_h.float()).abs()
+    assert (diff <= 2 ** -7 * want_h.float().abs() + 1e-6).all()
+    L2 = synth.make_layer(*synth.WORKLOADS["ffn_w2_m4352_k10240_n3840"],
+                          seed=synth.workload_seed("ffn_w2_m4352_k10240_n3840"))
+    r2 = H.gpu_layer(L2, x_override=h)
+    rows = H.sample_rows(L2.M, 24, seed=2)
+    y_ref, q_ref, a_ref, _ = H.oracle_y(L2, rows=rows, x=hd)
+    H.assert_quant_exact(r2["qact"][rows], r2["ascales"][rows], q_ref, a_ref, "w2 quant")
+    H.assert_y_close(r2["y"][rows], y_ref, "w2")
+
+
+def test_silu_mul_tail_and_values():
+    s = H.svdq()
+    g = torch.Generator().manual_seed(3)
+    for n in (1, 7, 8, 9, 1000, 4097):
+        a = torch.randn(n, generator=g).to(torch.bfloat16)
+        b = torch.randn(n, generator=g).to(torch.bfloat16)
+        out = s.silu_mul(a.cuda(), b.cuda()).cpu()
+        want = (a.float() * torch.sigmoid(a.float()) * b.float())
+        assert ((out.float() - want).abs() <= 2 ** -7 * want.abs() + 1e-6).all(), n
