@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="qkv_m4352_k3840_n11520")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffer) measurement")
     return ap.parse_args(argv)
 
 
@@ -282,7 +284,7 @@ def bench_ours(args, world, rank, local):
     traffic = load_traffic("w4a4_linear_kernel")
 
     # end to end through the public API with host buffers
-    e2e = bench_e2e(args, svdq, sets[0], dev, M, K, N, world)
+    e2e = None if args.no_e2e else bench_e2e(args, svdq, sets[0], dev, M, K, N, world)
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
