@@ -71,13 +71,31 @@ def load_peaks():
             "fallback"
 
 
+KERNEL_SOURCES = {
+    "w4a4_linear_kernel": "kg_w4a4_linear.cuh",
+    "quantize_act_kernel": "kq_quantize_act.cuh",
+}
+
+
+def kernel_source_hash(kernel_key):
+    import hashlib
+    path = os.path.join(ROOT, "nvfp4_w4a4_quantized_smooth_b200", "csrc",
+                        KERNEL_SOURCES[kernel_key])
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
 def load_traffic(kernel_key):
-    """Per-launch DRAM bytes of a kernel from the committed ncu summary, if any."""
+    """Per-launch DRAM bytes (read + write) of a kernel from the committed ncu
+    summary, or None if there is none or the kernel source changed since the
+    counters were taken (each line carries the source hash it was taken at)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         for line in open(path):
             parts = line.split()
-            if len(parts) >= 2 and parts[0] == kernel_key:
+            if len(parts) >= 3 and parts[0] == kernel_key:
+                if parts[2] != kernel_source_hash(kernel_key):
+                    return None
                 return float(parts[1])
     except OSError:
         pass
