@@ -142,6 +142,12 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
 
 /* ---- helpers ------------------------------------------------------------ */
 
+/* Launch shape svdq_quantize_act uses on the current device for an [M, K]
+ * input: rows per CTA (*bm, a multiple of 32 up to 128) and the number of
+ * CTAs of a thread-block cluster that split K (*split, 1..8).  Chosen so the
+ * whole grid is resident at once.  For inspection and tests; needs a device. */
+int svdq_quantize_plan(int M, int K, int* bm, int* split);
+
 /* Inverse of the tile order, for tests and inspection: tiled scales of
  * `rows` rows (M for activations, N for weights) -> out [rows, K/16]
  * bytes, device.  For weights this is the transpose of the on-disk

@@ -20,8 +20,12 @@
 //               tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64)
 //               into the main accumulator, then tcgen05.mma kind::f16
 //               (bf16, K=16) for L @ proj_up^T into a second accumulator.
-//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld), fp32
-//               acc * wtscale * wcscales + lowrank + bias, bf16 stores.
+//   warps 2..9  epilogue (two warps per TMEM lane quarter, one per half
+//               of the 256 columns): stage the tile's wcscales / bias in
+//               shared memory while the MMAs run, then TMEM -> registers
+//               (tcgen05.ld), fp32 acc * wtscale * wcscales + lowrank + bias,
+//               packed to bf16 in registers; TMEM is released before the
+//               global stores, so the stores overlap the next tile's MMAs.
 // TMEM map (512 columns, fp32): main accumulator [0, 256), low-rank
 // accumulator [256, 512); the per-step scale factors live in [256, 304)
 // while the main K loop runs (the low-rank MMAs start only after every main
@@ -52,8 +56,10 @@ constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr uint32_t LR_TX = LR_A_BYTES + LR_B_BYTES;
 constexpr uint32_t RING_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES);
 constexpr uint32_t BAR_BYTES = 128;
-constexpr uint32_t SMEM_BYTES = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
-constexpr int NUM_THREADS = 192;
+constexpr uint32_t COLV_BYTES = 2 * 2 * BN * 4;      // wcscales, bias (fp32), 2 tile buffers
+constexpr uint32_t SMEM_BYTES = RING_BYTES + COLV_BYTES + BAR_BYTES + 1024;  // + alignment
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0;
 constexpr uint32_t TM_LR = 256;
@@ -102,7 +108,8 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
   const uint32_t s_b = s_a + STAGES * A_BYTES;
   const uint32_t s_sfa = s_b + STAGES * B_BYTES;
   const uint32_t s_sfb = s_sfa + STAGES * SFA_BYTES;
-  const uint32_t s_bar = s_sfb + STAGES * SFB_BYTES;
+  const uint32_t s_colv = s_sfb + STAGES * SFB_BYTES;
+  const uint32_t s_bar = s_colv + COLV_BYTES;
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
   const uint32_t tmem_full_bar = s_bar + 16u * STAGES;
@@ -125,7 +132,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(tmem_full_bar, 1);
-    mbar_init(tmem_empty_bar, 4);
+    mbar_init(tmem_empty_bar, NUM_EPI_WARPS);
     mbar_init(drain_bar, 1);
     mbar_init(final_bar, 1);
     fence_mbar_init();
@@ -263,57 +270,71 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
     }
   } else {
     // -------------------------------------------------------- epilogue --
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;    // which 128 of the tile's 256 columns
+    const int et = threadIdx.x - 64;     // 0..255
     const float alpha = __bfloat162float(p.wtscale[0]);
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    float* colv = reinterpret_cast<float*>(smem + (s_colv - s_a));
     uint32_t tc = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int mb = t % p.m_tiles;
       const int nb = t / p.m_tiles;
+      // Per-column factors of this tile -> shared memory (double buffered by
+      // tile parity), loaded while the tile's MMAs are still running.
+      float* wc_s = colv + (tc & 1u) * (2 * BN);
+      float* bs_s = wc_s + BN;
+      {
+        const int n = nb * BN + et;
+        float wcv = 0.f, bsv = 0.f;
+        if (n < p.N) {
+          wcv = __bfloat162float(p.wcscales[n]);
+          if (p.bias != nullptr) bsv = __bfloat162float(p.bias[n]);
+        }
+        wc_s[et] = wcv * alpha;
+        bs_s[et] = bsv;
+      }
+      named_bar_sync(2, 32 * NUM_EPI_WARPS);
       if (!__all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI))) break;
       tc_fence_after();
       const int row = mb * BM + q * 32 + lane;
-      const bool row_ok = row < p.M;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t acc[32], lr[32];
-        tmem_ld_32x32b_x32(lane_base + TM_ACC + 32 * c, acc);
-        tmem_ld_32x32b_x32(lane_base + TM_LR + 32 * c, lr);
+      uint32_t out[4][16];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int col = half * 128 + 16 * c;
+        uint32_t acc[16], lr[16];
+        tmem_ld_32x32b_x16(lane_base + TM_ACC + col, acc);
+        tmem_ld_32x32b_x16(lane_base + TM_LR + col, lr);
         tmem_ld_wait();
-        const int n0 = nb * BN + 32 * c;
-        if (row_ok && n0 < p.N) {
-          const uint4* wc_src = reinterpret_cast<const uint4*>(p.wcscales + n0);
-          const uint4* b_src = reinterpret_cast<const uint4*>(p.bias + n0);
-          uint32_t out[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            float wc[8], bs[8];
-            unpack_bf16x8(__ldg(wc_src + v), wc);
-            if (p.bias != nullptr) {
-              unpack_bf16x8(__ldg(b_src + v), bs);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) bs[i] = 0.f;
-            }
-            float o[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float a = __uint_as_float(acc[8 * v + i]);
-              const float l = __uint_as_float(lr[8 * v + i]);
-              o[i] = fmaf(a * alpha, wc[i], l + bs[i]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) out[4 * v + i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(row) * p.ldy + n0);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+        for (int i = 0; i < 8; ++i) {
+          const float2 w2 = *reinterpret_cast<const float2*>(wc_s + col + 2 * i);
+          const float2 b2 = *reinterpret_cast<const float2*>(bs_s + col + 2 * i);
+          const float o0 = fmaf(__uint_as_float(acc[2 * i]), w2.x,
+                                __uint_as_float(lr[2 * i]) + b2.x);
+          const float o1 = fmaf(__uint_as_float(acc[2 * i + 1]), w2.y,
+                                __uint_as_float(lr[2 * i + 1]) + b2.y);
+          out[c >> 1][8 * (c & 1) + i] = pack_bf16x2(o0, o1);
         }
       }
+      // TMEM is free for the next tile as soon as every warp has its values.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tmem_empty_bar);
+      if (row < p.M) {
+        __nv_bfloat16* yrow = p.y + static_cast<size_t>(row) * p.ldy;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int n0 = nb * BN + half * 128 + 32 * c;
+          if (n0 < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(out[c][4 * v], out[c][4 * v + 1], out[c][4 * v + 2],
+                                  out[c][4 * v + 3]);
+          }
+        }
+      }
     }
   }
 

@@ -7,30 +7,37 @@
 // E2M1 elements, as the card's first paragraph states; rounding to
 // nearest-even with saturation):
 //   v = x * smooth                  exact in fp32 (bf16 x bf16)
-//   s = e4m3(amax|v| / 6)           fp32 division (correctly rounded), then
-//                                   the hardware RNE/satfinite conversion
-//   q = E2M1(v / s)                 quotient by reciprocal + one FMA
-//                                   residual correction, then the hardware
-//                                   RNE/satfinite conversion
-// Both roundings equal exact rational rounding: a bf16 x bf16 product has
-// at most 16 significant bits, every e4m3 midpoint x 6 and every E2M1
-// midpoint x s has at most 7, so a quotient that is not exactly on a
-// midpoint lies at least 2^-16 (relative) away from it, far more than the
-// fp32 error; a quotient exactly on a midpoint is representable, and the
-// residual step (r = RN(1/s), q0 = RN(v r), e = v - q0 s exact by FMA,
-// q = RN(q0 + e r); Markstein, IBM J. Res. Dev. 34(1), 1990) returns it
-// exactly, so the conversion sees the tie.
+//   s = e4m3(amax|v| / 6)           quotient, then the hardware RNE /
+//                                   satfinite conversion
+//   q = E2M1(v / s)                 quotient, then the hardware RNE /
+//                                   satfinite conversion
+// Each quotient a / b is formed as r = 1/b (reciprocal), q0 = a r, then one
+// residual step e = a - q0 b (exact by FMA), q = q0 + e r (Markstein, IBM J.
+// Res. Dev. 34(1), 1990).  Rounding that q equals rounding the exact
+// quotient: a bf16 x bf16 product has at most 16 significant bits, and
+// every e4m3 midpoint x 6 and every E2M1 midpoint x s at most 7, so a
+// quotient that is not exactly a midpoint lies at least 2^-16 (relative)
+// from it, far more than q's error (a few ulps of fp32); a quotient that is
+// exactly a midpoint is representable and the residual step returns it
+// exactly (|1 - b r| <= 2^-22 makes the step's error far below half an
+// ulp), so the conversion sees the tie.  A scale that rounds to zero gives
+// r = 0 and therefore signed zero codes.
 //
-// Layout of one CTA (128 rows x a K range, 10 warps):
-//   warp 0      TMA producer: x tile [128 rows x 64 k] bf16 (128-byte
-//               swizzle) and proj_down rows [64 k x 128 r] (two 64-column
-//               boxes) into a 4-stage ring.
-//   warp 1      TMEM owner, MMA issuer: L[128 x 128] += x_tile x pd_chunk
-//               with tcgen05.mma kind::f16 (M=128, N=128, K=16), A K-major,
-//               B MN-major, fp32 accumulator in 128 TMEM columns.
-//   warps 2..9  quantize the same shared-memory x tile (2 groups per
-//               thread per stage), write packed codes and tiled scales;
-//               afterwards read L out of TMEM.
+// CTA layout: a tile of BM rows (32..128) over a K range, 18 warps.
+//   warp 0      TMA producer: per stage of 128 k, the x tile as two
+//               [BM rows x 64 k] bf16 boxes (128-byte swizzle), proj_down
+//               rows [128 k x 128 r] (four 64 x 64 boxes) and the 128 smooth
+//               values, into a ring of stages.
+//   warp 1      TMEM owner, MMA issuer.  The low-rank product is computed
+//               transposed, L^T[128 x BM] += proj_down_chunk^T x_tile^T:
+//               tcgen05.mma kind::f16, M = 128 (= R), N = BM, K = 16;
+//               A (proj_down) MN-major, B (x tile) K-major, fp32 in BM
+//               TMEM columns.  So BM is free (multiple of 32) while the
+//               accumulator keeps the full 128-lane layout.
+//   warps 2..17 quantize the same shared-memory x tile (four warps per
+//               scheduler, one 16-element group per thread per stage for
+//               BM = 64), write packed codes and tiled scales; afterwards
+//               read L^T out of TMEM.
 // The K range is split over a thread-block cluster of `split` CTAs; the
 // partial L tiles are summed through distributed shared memory in rank
 // order (deterministic) and written once as bf16.
@@ -45,24 +52,43 @@
 namespace svdq {
 namespace kq {
 
-constexpr int BM = 128;               // rows per CTA
-constexpr int BKE = 64;               // k per stage
-constexpr int R = 128;                // rank (MMA N)
-constexpr int STAGES = 4;
-constexpr uint32_t X_BYTES = BM * BKE * 2;         // 16 KB
-constexpr uint32_t PD_BYTES = BKE * R * 2;         // 16 KB
-constexpr uint32_t PD_HALF = PD_BYTES / 2;         // one 64-column box
-constexpr uint32_t STAGE_BYTES = X_BYTES + PD_BYTES;
-constexpr int NUM_QWARPS = 8;
-constexpr int NUM_QTHREADS = NUM_QWARPS * 32;      // 256
-constexpr int NUM_THREADS = 64 + NUM_QTHREADS;     // 320
-constexpr uint32_t BAR_BYTES = 128;
-constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-constexpr uint32_t TMEM_COLS = 128;
-constexpr int PART_STRIDE = 132;  // floats per row of the partial-L buffer
-static_assert(BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partial buffer fits the ring");
+constexpr int R = 128;                 // rank (MMA M)
+constexpr int BKE = 64;                // k per chunk (one 128-byte swizzled box row)
+constexpr int CPS = 2;                 // chunks per stage
+constexpr int MAX_BM = 128;
+constexpr int MAX_STAGES = 6;
+constexpr uint32_t PD_BOX = 64 * 64 * 2;          // [64 k x 64 r] bf16 box, 8 KB
+constexpr uint32_t PD_CHUNK = 2 * PD_BOX;         // one chunk of proj_down, 16 KB
+constexpr uint32_t PD_BYTES = CPS * PD_CHUNK;     // 32 KB per stage
+constexpr uint32_t SMOOTH_CHUNK = BKE * 2;        // 128 B
+constexpr uint32_t SMOOTH_BYTES = CPS * SMOOTH_CHUNK;
+constexpr int NUM_QWARPS = 16;
+constexpr int NUM_QTHREADS = NUM_QWARPS * 32;
+constexpr int NUM_THREADS = 64 + NUM_QTHREADS;
+constexpr uint32_t BAR_BYTES = 256;
+constexpr uint32_t SMEM_BUDGET = 227 * 1024;
+constexpr int PART_STRIDE = R + 4;  // floats per row m of the partial-L buffer
 
 constexpr uint32_t SITE_PROD = 0x20, SITE_MMA = 0x21, SITE_QUANT = 0x22, SITE_LFULL = 0x23;
+
+__host__ __device__ constexpr uint32_t x_chunk(int bm) { return static_cast<uint32_t>(bm) * 128u; }
+__host__ __device__ constexpr uint32_t x_bytes(int bm) { return CPS * x_chunk(bm); }
+__host__ __device__ constexpr uint32_t stage_bytes(int bm) {
+  return (x_bytes(bm) + PD_BYTES + SMOOTH_BYTES + 1023u) & ~1023u;
+}
+__host__ __device__ constexpr int num_stages(int bm) {
+  return (SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm) < MAX_STAGES
+             ? static_cast<int>((SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm))
+             : MAX_STAGES;
+}
+__host__ __device__ constexpr uint32_t smem_bytes(int bm) {
+  return num_stages(bm) * stage_bytes(bm) + BAR_BYTES + 1024;
+}
+__host__ __device__ constexpr uint32_t tmem_cols(int bm) {
+  return bm <= 32 ? 32u : bm <= 64 ? 64u : 128u;
+}
+static_assert(MAX_BM * PART_STRIDE * 4 <= 2 * stage_bytes(MAX_BM), "partial buffer fits the ring");
+static_assert(num_stages(32) >= 2 && num_stages(MAX_BM) >= 2, "at least two stages");
 
 struct Params {
   const __nv_bfloat16* smooth;
@@ -72,6 +98,7 @@ struct Params {
   int M, K;
   int chunks;  // K / 64
   int split;   // CTAs per cluster along K
+  int bm;      // rows per CTA (multiple of 32, <= 128)
 };
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
@@ -82,69 +109,112 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// Packed pairs of fp32 (lo in the low word) and their arithmetic.
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// bf16 pair word -> packed fp32 pair (element 2i in the low word).
+__device__ __forceinline__ uint64_t bf16x2_to_pk(uint32_t w) {
+  return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// One 16-element group: x (8 bf16x2 words), smooth (8 bf16x2 words) ->
+// 16 E2M1 codes (element 0 in the lowest nibble) and the e4m3 scale byte.
+__device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8], const uint32_t (&sw)[8],
+                                                   uint32_t& scale_byte) {
+  uint64_t v[8];
+  float m8[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  for (int i = 0; i < 8; ++i) {
+    v[i] = mul2(bf16x2_to_pk(xw[i]), bf16x2_to_pk(sw[i]));
+    float lo, hi;
+    upk(v[i], lo, hi);
+    m8[i] = fmaxf(fabsf(lo), fabsf(hi));
   }
-}
-
-// Quantize one 16-element group: v[16] (x * smooth, exact) -> 16 E2M1
-// codes (64 bits, element 0 in the lowest nibble) and the e4m3 scale byte.
-__device__ __forceinline__ uint64_t quantize_group(const float (&v)[16], uint32_t& scale_byte) {
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  const uint32_t sc = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xFFu;
+  // max is exact, so a tree gives the same amax with a short dependency chain
+  const float amax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+  // amax / 6 with one residual step; r6 = RN(1/6).
+  const float r6 = __uint_as_float(0x3E2AAAABu);
+  const float a0 = amax * r6;
+  const float a6 = fmaf(fmaf(-a0, 6.0f, amax), r6, a0);
+  const uint32_t sc = cvt_e4m3x2(a6, 0.0f) & 0xFFu;
   scale_byte = sc;
   const float d = e4m3_to_f32(sc);
-  if (d == 0.0f) {
-    // Every element rounds to zero; keep each element's sign.
-    uint64_t codes = 0;
+  const float r = d > 0.0f ? rcp_approx(d) : 0.0f;
+  const uint64_t r2 = pk(r, r);
+  const uint64_t nd2 = pk(-d, -d);
+  float q[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      codes |= static_cast<uint64_t>(__float_as_uint(v[i]) >> 31) << (4 * i + 3);
-    return codes;
+  for (int i = 0; i < 8; ++i) {
+    const uint64_t q0 = mul2(v[i], r2);
+    const uint64_t e = fma2(q0, nd2, v[i]);
+    const uint64_t q1 = fma2(e, r2, q0);
+    float lo, hi, vlo, vhi;
+    upk(q1, lo, hi);
+    upk(v[i], vlo, vhi);
+    // The residual step turns a quotient of -0 into +0: restore v's sign.
+    q[2 * i] = __uint_as_float((__float_as_uint(lo) & 0x7FFFFFFFu) |
+                               (__float_as_uint(vlo) & 0x80000000u));
+    q[2 * i + 1] = __uint_as_float((__float_as_uint(hi) & 0x7FFFFFFFu) |
+                                   (__float_as_uint(vhi) & 0x80000000u));
   }
-  const float r = __frcp_rn(d);
-  float lo[8], hi[8];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float q0 = v[i] * r;
-    const float e = fmaf(-q0, d, v[i]);
-    float q = fmaf(e, r, q0);
-    // The correction turns a quotient of -0 into +0: restore v's sign.
-    q = __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(v[i]) & 0x80000000u));
-    if (i < 8) lo[i] = q; else hi[i - 8] = q;
-  }
-  return static_cast<uint64_t>(cvt_e2m1x8(lo)) | (static_cast<uint64_t>(cvt_e2m1x8(hi)) << 32);
+  const float(&qlo)[8] = *reinterpret_cast<const float(*)[8]>(q);
+  const float(&qhi)[8] = *reinterpret_cast<const float(*)[8]>(q + 8);
+  return static_cast<uint64_t>(cvt_e2m1x8(qlo)) | (static_cast<uint64_t>(cvt_e2m1x8(qhi)) << 32);
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] bf16
-                    const __grid_constant__ CUtensorMap tm_pd,   // proj_down [K, 128] bf16
+quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] bf16, box {64, bm}
+                    const __grid_constant__ CUtensorMap tm_pd,   // proj_down [K, 128], box {64, 64}
                     const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int bm = p.bm;
+  const uint32_t sbytes = stage_bytes(bm);
+  const uint32_t nst = static_cast<uint32_t>(num_stages(bm));
   const uint32_t s_ring = smem_u32(smem);
-  const uint32_t s_bar = s_ring + STAGES * STAGE_BYTES;
-  auto s_x = [&](uint32_t s) { return s_ring + s * STAGE_BYTES; };
-  auto s_pd = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + X_BYTES; };
+  const uint32_t s_bar = s_ring + nst * sbytes;
+  // Stage layout: x chunks [CPS][bm rows x 128 B], proj_down chunks
+  // [CPS][r half][64 k x 128 B], smooth chunks [CPS][128 B].
+  auto s_x = [&](uint32_t s, int c) { return s_ring + s * sbytes + c * x_chunk(bm); };
+  auto s_pd = [&](uint32_t s, int c) { return s_ring + s * sbytes + x_bytes(bm) + c * PD_CHUNK; };
+  auto s_sm = [&](uint32_t s, int c) {
+    return s_ring + s * sbytes + x_bytes(bm) + PD_BYTES + c * SMOOTH_CHUNK;
+  };
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
-  auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
-  const uint32_t lfull_bar = s_bar + 16u * STAGES;
+  auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (MAX_STAGES + s); };
+  const uint32_t lfull_bar = s_bar + 16u * MAX_STAGES;
   const uint32_t final_bar = lfull_bar + 8u;
   const uint32_t tmem_slot = lfull_bar + 16u;
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
+  const uint32_t ncols = tmem_cols(bm);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -152,12 +222,14 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   const int rank = blockIdx.x;  // == rank in the cluster (cluster dims = (split, 1, 1))
   const int c_begin = rank * p.chunks / p.split;
   const int c_end = (rank + 1) * p.chunks / p.split;
-  const int nchunks = c_end - c_begin;  // >= 1 (host guarantees split <= chunks)
+  // >= 1 chunk per CTA (host guarantees split <= chunks); stages of CPS
+  // chunks, the last one possibly partial.
+  const int nstages = (c_end - c_begin + CPS - 1) / CPS;
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_pd);
-    for (uint32_t s = 0; s < STAGES; ++s) {
+    for (uint32_t s = 0; s < nst; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1 + NUM_QWARPS);
     }
@@ -166,7 +238,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_alloc(tmem_slot, ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -181,48 +253,57 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
       // ------------------------------------------------------ producer --
       int i = 0;
       bool ok = true;
-      for (; i < nchunks; ++i) {
-        const uint32_t s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1u;
+      for (; i < nstages; ++i) {
+        const uint32_t s = static_cast<uint32_t>(i) % nst;
+        const uint32_t ph = (static_cast<uint32_t>(i) / nst) & 1u;
         if (!svdq_wait(empty_bar(s), ph ^ 1u, SITE_PROD)) {
           ok = false;
           break;
         }
-        const int kc = c_begin + i;
-        mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
-        tma_load_2d(s_x(s), &tm_x, kc * BKE, mb * BM, full_bar(s));
-        tma_load_2d(s_pd(s), &tm_pd, 0, kc * BKE, full_bar(s));
-        tma_load_2d(s_pd(s) + PD_HALF, &tm_pd, 64, kc * BKE, full_bar(s));
+        const int kc0 = c_begin + CPS * i;
+        const int nc = c_end - kc0 < CPS ? c_end - kc0 : CPS;
+        mbar_arrive_expect_tx(full_bar(s), nc * (x_chunk(bm) + PD_CHUNK + SMOOTH_CHUNK));
+        for (int c = 0; c < nc; ++c) {
+          const int kc = kc0 + c;
+          tma_load_2d(s_x(s, c), &tm_x, kc * BKE, mb * bm, full_bar(s));
+          tma_load_2d(s_pd(s, c), &tm_pd, 0, kc * BKE, full_bar(s));
+          tma_load_2d(s_pd(s, c) + PD_BOX, &tm_pd, 64, kc * BKE, full_bar(s));
+          bulk_load(s_sm(s, c), p.smooth + kc * BKE, SMOOTH_CHUNK, full_bar(s));
+        }
       }
       if (!ok) {
-        const int n = i < STAGES ? i : STAGES;
+        const int n = i < static_cast<int>(nst) ? i : static_cast<int>(nst);
         for (int j = 0; j < n; ++j) {
-          const int jt = i - 1 - j;
-          drain_wait(full_bar(jt % STAGES), (jt / STAGES) & 1u, 50000000ull);
+          const uint32_t jt = static_cast<uint32_t>(i - 1 - j);
+          drain_wait(full_bar(jt % nst), (jt / nst) & 1u, 50000000ull);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------- MMA issuer --
-      const uint32_t idesc = idesc_bf16_f32(BM, R, 0, 1);
+      // L^T[r, m] += sum_k proj_down[k, r] x[m, k]: A = proj_down chunk
+      // (MN-major: r contiguous; the two 64-r halves are 8 KB apart, 8-row
+      // k groups 1 KB apart), B = x chunk (K-major, 128-byte rows).
+      const uint32_t idesc = idesc_bf16_f32(R, static_cast<uint32_t>(bm), 1, 0);
       bool ok = true;
-      for (int i = 0; i < nchunks; ++i) {
-        const uint32_t s = i % STAGES;
-        const uint32_t ph = (i / STAGES) & 1u;
+      for (int i = 0; i < nstages; ++i) {
+        const uint32_t s = static_cast<uint32_t>(i) % nst;
+        const uint32_t ph = (static_cast<uint32_t>(i) / nst) & 1u;
         if (!svdq_wait(full_bar(s), ph, SITE_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const int kc0 = c_begin + CPS * i;
+        const int nc = c_end - kc0 < CPS ? c_end - kc0 : CPS;
+        for (int c = 0; c < nc; ++c) {
 #pragma unroll
-        for (int kk = 0; kk < BKE / 16; ++kk) {
-          // A: 16 k of the x tile = 32 bytes along the swizzled row.
-          // B: 16 k rows of proj_down = 2 swizzle atoms of 8 rows (1 KB
-          //    each); the two 64-column halves are 8 KB apart.
-          mma_f16(tmem_base, smem_desc(s_x(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B),
-                  smem_desc(s_pd(s) + 2048 * kk, PD_HALF, 1024, kLayoutSwizzle128B), idesc,
-                  (i | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BKE / 16; ++kk) {
+            mma_f16(tmem_base, smem_desc(s_pd(s, c) + 2048 * kk, PD_BOX, 1024, kLayoutSwizzle128B),
+                    smem_desc(s_x(s, c) + 32 * kk, 16, 1024, kLayoutSwizzle128B), idesc,
+                    (i | c | kk) != 0 ? 1u : 0u);
+          }
         }
         tc_commit(empty_bar(s));
       }
@@ -234,50 +315,53 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
     // -------------------------------------------------------- quantizers --
     const int qt = threadIdx.x - 64;
     const int half_k = p.K / 2;
+    const int rows_pad = (p.M + 127) & ~127;   // rows the tiled scale buffer holds
     bool ok = true;
-    for (int i = 0; i < nchunks; ++i) {
-      const uint32_t s = i % STAGES;
-      const uint32_t ph = (i / STAGES) & 1u;
+    for (int i = 0; i < nstages; ++i) {
+      const uint32_t s = static_cast<uint32_t>(i) % nst;
+      const uint32_t ph = (static_cast<uint32_t>(i) / nst) & 1u;
       if (!__all_sync(0xFFFFFFFFu, svdq_wait(full_bar(s), ph, SITE_QUANT))) {
         ok = false;
         break;
       }
-      const int kc = c_begin + i;
-#pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        const int gi = pass * NUM_QTHREADS + qt;
-        const int r = gi >> 2;  // row in the tile
-        const int g = gi & 3;   // group of 16 within the 64-wide chunk
-        const uint32_t row_addr = s_x(s) + r * 128;
-        const uint4 xa = ld_shared_v4(row_addr + (((2 * g) ^ (r & 7)) << 4));
-        const uint4 xb = ld_shared_v4(row_addr + (((2 * g + 1) ^ (r & 7)) << 4));
-        const uint4* sp = reinterpret_cast<const uint4*>(p.smooth + kc * BKE + g * 16);
-        const uint4 sa = __ldg(sp);
-        const uint4 sb = __ldg(sp + 1);
-        float xv[16], sv[16], v[16];
-        bf16x8_to_f32(xa, xv);
-        bf16x8_to_f32(xb, xv + 8);
-        bf16x8_to_f32(sa, sv);
-        bf16x8_to_f32(sb, sv + 8);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = xv[e] * sv[e];
-        uint32_t scale;
-        const uint64_t codes = quantize_group(v, scale);
-        const int row = mb * BM + r;
-        if (row < p.M) {
-          uint2* dst = reinterpret_cast<uint2*>(p.qact + static_cast<size_t>(row) * half_k +
-                                                kc * (BKE / 2) + g * 8);
-          *dst = make_uint2(static_cast<uint32_t>(codes), static_cast<uint32_t>(codes >> 32));
+      const int kc0 = c_begin + CPS * i;
+      const int nc = c_end - kc0 < CPS ? c_end - kc0 : CPS;
+      // bm rows x (4 nc) groups; lanes 8j..8j+7 take one row's 8 groups
+      // (chunk c = lane / 4 % 2, group g = lane % 4), whole warps together.
+      for (int gi = qt; gi < bm * 4 * CPS; gi += NUM_QTHREADS) {
+        const int r = gi >> 3;       // row in the tile
+        const int c = (gi >> 2) & 1; // chunk within the stage
+        const int g = gi & 3;        // group of 16 within the chunk
+        const bool active = c < nc;     // the stage's second chunk may be absent
+        const int row = mb * bm + r;
+        const int kc = kc0 + c;
+        uint32_t scale = 0;
+        if (active) {
+          const uint32_t row_addr = s_x(s, c) + r * 128;
+          const uint4 xa = ld_shared_v4(row_addr + (((2 * g) ^ (r & 7)) << 4));
+          const uint4 xb = ld_shared_v4(row_addr + (((2 * g + 1) ^ (r & 7)) << 4));
+          const uint4 sa = ld_shared_v4(s_sm(s, c) + g * 32);
+          const uint4 sb = ld_shared_v4(s_sm(s, c) + g * 32 + 16);
+          const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+          const uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+          const uint64_t codes = quantize_group(xw, sw, scale);
+          if (row < p.M) {
+            uint2* dst = reinterpret_cast<uint2*>(p.qact + static_cast<size_t>(row) * half_k +
+                                                  kc * (BKE / 2) + g * 8);
+            *dst = make_uint2(static_cast<uint32_t>(codes), static_cast<uint32_t>(codes >> 32));
+          }
         }
         // Tiled scales: 512-byte block per (128 rows, 4 groups); byte
-        // (r % 32) * 16 + (r / 32) * 4 + g.  Lanes 4i..4i+3 hold one row.
+        // (row % 32) * 16 + ((row % 128) / 32) * 4 + g.  Lanes 4j..4j+3 hold
+        // one row's four groups of one chunk; every lane takes part in the
+        // shuffles.
         uint32_t w = scale << (8 * g);
         w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
         w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
-        if (g == 0) {
+        if (active && g == 0 && row < rows_pad) {
           uint32_t* sdst = reinterpret_cast<uint32_t*>(
-              p.ascales_tiled + (static_cast<size_t>(mb) * p.chunks + kc) * 512 + (r & 31) * 16 +
-              (r >> 5) * 4);
+              p.ascales_tiled + (static_cast<size_t>(row >> 7) * p.chunks + kc) * 512 +
+              (row & 31) * 16 + ((row & 127) >> 5) * 4);
           *sdst = w;
         }
       }
@@ -289,69 +373,68 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   }
 
   // --------------------------------------------------- low-rank readout --
-  // Quantizer warp w reads TMEM lane quarter (w % 4), columns [64 h, 64 h + 64).
+  // TMEM holds L^T: lane r, column m.  The four quantizer warps of lane
+  // quarter (w % 4) read its columns in four slices of bm / 4.
   const bool is_q = warp >= 2;
   const int lq = warp & 3;
-  const int hcol = (warp - 2) >> 2;
-  const int r_out = lq * 32 + lane;
-  const int row_out = mb * BM + r_out;
+  const int slice = (warp - 2) >> 2;
+  const int r_lane = lq * 32 + lane;
+  const int cw = bm >> 2;  // columns per warp (multiple of 8)
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lq * 32) << 16);
   if (p.split == 1) {
     if (is_q && l_ready) {
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t acc[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(lq * 32) << 16) + 64 * hcol + 32 * c,
-                           acc);
+      for (int c0 = slice * cw; c0 < (slice + 1) * cw; c0 += 8) {
+        uint32_t v[8];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+              "=r"(v[6]), "=r"(v[7])
+            : "r"(lane_addr + c0)
+            : "memory");
         tmem_ld_wait();
-        if (row_out < p.M) {
-          uint4* dst = reinterpret_cast<uint4*>(p.lowrank + static_cast<size_t>(row_out) * R +
-                                                64 * hcol + 32 * c);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(acc[8 * v + 2 * i]),
-                                                        __uint_as_float(acc[8 * v + 2 * i + 1]));
-              w[i] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+        for (int j = 0; j < 8; ++j) {
+          const int row = mb * bm + c0 + j;
+          if (row < p.M)
+            p.lowrank[static_cast<size_t>(row) * R + r_lane] =
+                __float2bfloat16_rn(__uint_as_float(v[j]));
         }
       }
     }
   } else {
     // Partial sums: every quantizer warp has finished with the ring before
-    // any of them overwrites it with its fp32 partial L rows.
+    // any of them overwrites it with its fp32 partial (row-major [m][r]).
     if (is_q) {
       named_bar_sync(1, NUM_QTHREADS);
       if (l_ready) {
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t acc[32];
-          tmem_ld_32x32b_x32(
-              tmem_base + (static_cast<uint32_t>(lq * 32) << 16) + 64 * hcol + 32 * c, acc);
+        for (int c0 = slice * cw; c0 < (slice + 1) * cw; c0 += 8) {
+          uint32_t v[8];
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                "=r"(v[6]), "=r"(v[7])
+              : "r"(lane_addr + c0)
+              : "memory");
           tmem_ld_wait();
-          const uint32_t base = s_ring + (r_out * PART_STRIDE + 64 * hcol + 32 * c) * 4;
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            st_shared_v4(base + 16 * v, __uint_as_float(acc[4 * v]),
-                         __uint_as_float(acc[4 * v + 1]), __uint_as_float(acc[4 * v + 2]),
-                         __uint_as_float(acc[4 * v + 3]));
+          for (int j = 0; j < 8; ++j)
+            st_shared_f32(s_ring + ((c0 + j) * PART_STRIDE + r_lane) * 4, __uint_as_float(v[j]));
         }
       }
     }
     __syncwarp();
     cluster_sync_all();
     if (is_q && !error_raised()) {
-      const int rows_per = BM / p.split;
-      const int row0 = rank * rows_per;
-      for (int idx = threadIdx.x - 64; idx < rows_per * (R / 4); idx += NUM_QTHREADS) {
-        const int rr = row0 + idx / (R / 4);
-        const int c4 = idx % (R / 4);
-        const uint32_t off = s_ring + (rr * PART_STRIDE + 4 * c4) * 4;
+      // This rank sums its share of the bm x 32 float4 units over all ranks.
+      const int units = bm * (R / 4);
+      const int u0 = rank * units / p.split;
+      const int u1 = (rank + 1) * units / p.split;
+      for (int u = u0 + (threadIdx.x - 64); u < u1; u += NUM_QTHREADS) {
+        const int m = u / (R / 4);
+        const int c4 = u % (R / 4);
+        const uint32_t off = s_ring + (m * PART_STRIDE + 4 * c4) * 4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int src = 0; src < p.split; ++src) {
           const float4 t = ld_dsmem_f4(map_to_rank(off, src));
@@ -360,7 +443,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
           acc.z += t.z;
           acc.w += t.w;
         }
-        const int row = mb * BM + rr;
+        const int row = mb * bm + m;
         if (row < p.M) {
           __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
           __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
@@ -379,7 +462,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, ncols);
   }
 }
 

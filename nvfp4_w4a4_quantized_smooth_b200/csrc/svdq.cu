@@ -23,6 +23,9 @@ struct DeviceInfo {
   bool init = false;
   bool sm100 = false;
   int num_sms = 0;
+  // Max co-resident clusters of the activation kernel, by (bm / 32, split);
+  // -1 = not queried yet.
+  int kq_clusters[9][9];
 };
 
 std::mutex g_mu;
@@ -47,10 +50,12 @@ int device_setup(DeviceInfo** out) {
       return SVDQ_ERR_CUDA;
     d.sm100 = (major == 10 && minor == 0);
     d.num_sms = sms;
+    for (auto& row : d.kq_clusters)
+      for (int& v : row) v = -1;
     if (d.sm100) {
       if (cudaFuncSetAttribute(svdq::kq::quantize_act_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               svdq::kq::SMEM_BYTES) != cudaSuccess ||
+                               svdq::kq::SMEM_BUDGET) != cudaSuccess ||
           cudaFuncSetAttribute(svdq::kg::w4a4_linear_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                svdq::kg::SMEM_BYTES) != cudaSuccess)
@@ -98,6 +103,60 @@ int grid_for(size_t work, int threads, int num_sms) {
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return static_cast<int>(blocks);
+}
+
+
+// How many clusters of `split` activation-kernel CTAs with row tile `bm` can
+// be resident at once on this device (cached).
+int kq_max_clusters(DeviceInfo* d, int bm, int split) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int& slot = d->kq_clusters[bm / 32][split];
+  if (slot >= 0) return slot;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(split, 1024, 1);
+  cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = svdq::kq::smem_bytes(bm);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel),
+                                     &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  slot = n;
+  return n;
+}
+
+// Row tile and K split of the activation kernel: the single-wave grid
+// (m_tiles clusters of `split` CTAs, at most one CTA per SM, every cluster
+// co-resident) that occupies the most SMs; ties go to less row padding, then
+// to the larger row tile (less proj_down traffic per row).
+void kq_plan(DeviceInfo* d, int M, int chunks, int* bm_out, int* split_out) {
+  int best_bm = svdq::kq::MAX_BM, best_split = 1, best_score = -1, best_waste = 0;
+  for (int bm = svdq::kq::MAX_BM; bm >= 32; bm -= 32) {
+    const int m_tiles = (M + bm - 1) / bm;
+    const int waste = m_tiles * bm - M;
+    for (int split = 1; split <= 8 && split <= chunks; ++split) {
+      const int ctas = m_tiles * split;
+      if (ctas > d->num_sms) break;
+      if (m_tiles > kq_max_clusters(d, bm, split)) continue;
+      if (ctas > best_score || (ctas == best_score && waste < best_waste)) {
+        best_score = ctas;
+        best_waste = waste;
+        best_bm = bm;
+        best_split = split;
+      }
+    }
+  }
+  *bm_out = best_bm;        // no single-wave plan: largest tile, no split
+  *split_out = best_split;
 }
 
 }  // namespace
@@ -172,18 +231,17 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   DeviceInfo* d = nullptr;
   if (int st = device_setup(&d)) return st;
 
+  const int chunks = K / svdq::kq::BKE;
+  int bm = 0, split = 0;
+  kq_plan(d, M, chunks, &bm, &split);
+  const int m_tiles = (M + bm - 1) / bm;
+
   CUtensorMap tm_x, tm_pd;
   if (make_tmap(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, M, static_cast<uint64_t>(ldx) * 2,
-                svdq::kq::BKE, svdq::kq::BM) ||
+                svdq::kq::BKE, bm) ||
       make_tmap(&tm_pd, proj_down, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, K,
                 static_cast<uint64_t>(R) * 2, 64, svdq::kq::BKE))
     return SVDQ_ERR_CUDA;
-
-  const int m_tiles = (M + svdq::kq::BM - 1) / svdq::kq::BM;
-  const int chunks = K / svdq::kq::BKE;
-  // Split K over a cluster until the grid covers the SMs once.
-  int split = 1;
-  while (split < 8 && m_tiles * split * 2 <= d->num_sms && chunks >= split * 2) split *= 2;
 
   svdq::kq::Params p;
   p.smooth = reinterpret_cast<const __nv_bfloat16*>(smooth);
@@ -194,12 +252,13 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   p.K = K;
   p.chunks = chunks;
   p.split = split;
+  p.bm = bm;
 
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(split, m_tiles, 1);
   cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = svdq::kq::SMEM_BYTES;
+  cfg.dynamicSmemBytes = svdq::kq::smem_bytes(bm);
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -260,6 +319,16 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   svdq::kg::w4a4_linear_kernel<<<grid, svdq::kg::NUM_THREADS, svdq::kg::SMEM_BYTES,
                                  static_cast<cudaStream_t>(stream)>>>(tm_a, tm_b, tm_l, tm_p, p);
   return launch_status();
+}
+
+int svdq_quantize_plan(int M, int K, int* bm, int* split) {
+  if (!bm || !split) return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || K < 16 || K % 16) return SVDQ_ERR_SHAPE;
+  if (K % 64) return SVDQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  kq_plan(d, M, K / svdq::kq::BKE, bm, split);
+  return SVDQ_OK;
 }
 
 int svdq_unpack_scales(const void* scales_tiled, int rows, int K, uint8_t* out, void* stream) {

@@ -41,6 +41,7 @@ SIGNATURES = {
     "svdq_repack_weights": (_I, [_P, _I, _I, _P, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
     "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
+    "svdq_quantize_plan": (_I, [_I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "svdq_unpack_scales": (_I, [_P, _I, _I, _P, _P]),
     "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
     "svdq_check_device_error": (_I, [_P]),
@@ -173,6 +174,14 @@ def w4a4_linear(qact: torch.Tensor, ascales_tiled: torch.Tensor, lowrank: torch.
                                  _ptr(y), y.stride(0), _stream(stream)),
            "svdq_w4a4_linear")
     return y
+
+
+def quantize_plan(M: int, K: int):
+    """(rows per CTA, K split) svdq_quantize_act uses for [M, K] on this device."""
+    bm, split = _I(), _I()
+    _check(_lib.svdq_quantize_plan(M, K, ctypes.byref(bm), ctypes.byref(split)),
+           "svdq_quantize_plan")
+    return bm.value, split.value
 
 
 def unpack_scales(scales_tiled: torch.Tensor, rows: int, K: int, stream=None) -> torch.Tensor:

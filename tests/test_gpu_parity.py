@@ -59,7 +59,8 @@ def test_repack_rejects_sign_and_nan_scales(bad):
 # ----------------------------------------------------------- quantize ---
 
 @pytest.mark.parametrize("M,K", [(1, 64), (17, 128), (128, 512), (129, 512), (300, 192),
-                                 (64, 3840), (513, 1024), (16, 10240)])
+                                 (64, 3840), (513, 1024), (16, 10240), (100, 640), (1000, 448),
+                                 (2000, 256), (4352, 256)])
 def test_quantize_act_bit_exact_and_lowrank(M, K):
     s = H.svdq()
     L = synth.make_layer(M, K, 32, seed=M * 7 + K)
@@ -70,6 +71,19 @@ def test_quantize_act_bit_exact_and_lowrank(M, K):
                          f"M={M} K={K}")
     L_ref = ref.lowrank_down(H.bits(L.x), H.bits(L.proj_down))
     H.assert_lowrank_close(lr.cpu(), L_ref, f"M={M} K={K}")
+
+
+def test_quantize_plans_fit_one_wave():
+    # The launch plan keeps the grid resident at once and covers every row.
+    s = H.svdq()
+    for M in (1, 16, 64, 100, 256, 1024, 4352, 17408):
+        for K in (64, 512, 3840, 10240):
+            bm, split = s.quantize_plan(M, K)
+            assert bm % 32 == 0 and 32 <= bm <= 128, (M, K, bm)
+            assert 1 <= split <= min(8, K // 64), (M, K, split)
+            tiles = -(-M // bm)
+            if tiles * split > torch.cuda.get_device_properties(0).multi_processor_count:
+                assert split == 1 and bm == 128, (M, K, bm, split)
 
 
 def _golden_rows():
