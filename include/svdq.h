@@ -67,7 +67,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 1
+#define SVDQ_ABI_VERSION 2
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -77,7 +77,9 @@ int svdq_abi_version(void);
 size_t svdq_ascales_tiled_bytes(int M, int K);
 
 /* Tiled weight scales written by svdq_repack_weights for N output
- * channels: ceil(N/256)*2 * (K/64) blocks of 512 bytes.  0 on bad args. */
+ * channels: ceil(N/256)*2 * (K/64) blocks of 512 bytes.  0 on bad args.
+ * Block order: 256-row tile, then K block of 64, then 128-row half, so
+ * that the scales one GEMM tile needs for a run of K are contiguous. */
 size_t svdq_wscales_tiled_bytes(int N, int K);
 
 /* Low-rank activations L = x @ proj_down written by svdq_quantize_act:
@@ -143,16 +145,21 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
 /* ---- helpers ------------------------------------------------------------ */
 
 /* Launch shape svdq_quantize_act uses on the current device for an [M, K]
- * input: rows per CTA (*bm, a multiple of 32 up to 128) and the number of
+ * input: rows per CTA (*bm, a multiple of 32 up to 256) and the number of
  * CTAs of a thread-block cluster that split K (*split, 1..8).  Chosen so the
- * whole grid is resident at once.  For inspection and tests; needs a device. */
+ * whole grid is resident at once when it can be.  For inspection and tests;
+ * needs a device. */
 int svdq_quantize_plan(int M, int K, int* bm, int* split);
 
 /* Inverse of the tile order, for tests and inspection: tiled scales of
- * `rows` rows (M for activations, N for weights) -> out [rows, K/16]
- * bytes, device.  For weights this is the transpose of the on-disk
- * wscales [K/16, N]. */
-int svdq_unpack_scales(const void* scales_tiled, int rows, int K,
+ * `rows` rows -> out [rows, K/16] bytes, device.  `kind` says which order
+ * the buffer has: SVDQ_SCALES_ACT (written by svdq_quantize_act, rows = M)
+ * or SVDQ_SCALES_WEIGHT (written by svdq_repack_weights, rows = N; the
+ * result is then the transpose of the on-disk wscales [K/16, N]).  Any
+ * other kind gives SVDQ_ERR_INVALID_ARG. */
+#define SVDQ_SCALES_ACT 0
+#define SVDQ_SCALES_WEIGHT 1
+int svdq_unpack_scales(const void* scales_tiled, int rows, int K, int kind,
                        uint8_t* out, void* stream);
 
 /* out[i] = silu(a[i]) * b[i] in fp32, rounded to bf16; n elements.  Used

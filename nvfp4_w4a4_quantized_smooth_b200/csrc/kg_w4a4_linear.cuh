@@ -8,13 +8,14 @@
 // with L = x @ proj_down from the activation kernel, stored bf16.
 //
 // Design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: per K step of 256 it loads the A tile
-//               (qact, 128 rows x 128 B), the B tile (qweight, 256 rows x
-//               128 B), both 128-byte swizzled, and the matching scale
-//               blocks (bulk copies of the tiled scale buffers) into a
-//               4-stage shared-memory ring; after the K loop it loads the
-//               low-rank operands (L and proj_up, two K halves of 64)
-//               through the same ring.
+//   warp 0      TMA producer.  A ring of STAGES slots; a slot holds one K
+//               step of 256: the qact box (128 rows x 128 B, 128-byte
+//               swizzle), the qweight box (256 rows x 128 B) and one
+//               contiguous bulk copy each of the step's A and B scale
+//               blocks.  After the K steps of a tile, two more slots carry
+//               the low-rank operands, one 64-wide half of R each (L half
+//               in the A place, proj_up half in the B place), so they are
+//               prefetched like any other step.
 //   warp 1      TMEM owner and MMA issuer (one thread): copies the scale
 //               blocks smem -> TMEM (tcgen05.cp), issues
 //               tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64)
@@ -24,12 +25,14 @@
 //               of the 256 columns): stage the tile's wcscales / bias in
 //               shared memory while the MMAs run, then TMEM -> registers
 //               (tcgen05.ld), fp32 acc * wtscale * wcscales + lowrank + bias,
-//               packed to bf16 in registers; TMEM is released before the
-//               global stores, so the stores overlap the next tile's MMAs.
+//               packed to bf16.  TMEM is released to the next tile right
+//               after the reads; the bf16 rows then go through a per-warp
+//               swizzled shared-memory buffer to TMA tensor stores, which
+//               write whole rows asynchronously and clip the M / N edges.
 // TMEM map (512 columns, fp32): main accumulator [0, 256), low-rank
-// accumulator [256, 512); the per-step scale factors live in [256, 304)
-// while the main K loop runs (the low-rank MMAs start only after every main
-// MMA has completed).
+// accumulator [256, 512); the scale factors of the ring slots live in
+// [256, 400) while the main K loop runs (the low-rank MMAs start only after
+// every main MMA has completed).
 #pragma once
 
 #include <cuda.h>
@@ -45,26 +48,31 @@ constexpr int BM = 128;          // output rows per tile (MMA M)
 constexpr int BN = 256;          // output columns per tile (MMA N)
 constexpr int BK_BYTES = 128;    // K step: 256 FP4 values = 128 bytes per row
 constexpr int BK = 256;
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr uint32_t A_BYTES = BM * BK_BYTES;          // 16 KB
 constexpr uint32_t B_BYTES = BN * BK_BYTES;          // 32 KB
 constexpr uint32_t SFA_BYTES = 4 * 512;              // 128 rows x 16 scales
 constexpr uint32_t SFB_BYTES = 2 * 4 * 512;          // 256 rows x 16 scales
-constexpr uint32_t LR_A_BYTES = BM * 128;            // 128 rows x 64 bf16
-constexpr uint32_t LR_B_BYTES = BN * 128;            // 256 rows x 64 bf16
-constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr uint32_t LR_TX = LR_A_BYTES + LR_B_BYTES;
-constexpr uint32_t RING_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES);
-constexpr uint32_t BAR_BYTES = 128;
-constexpr uint32_t COLV_BYTES = 2 * 2 * BN * 4;      // wcscales, bias (fp32), 2 tile buffers
-constexpr uint32_t SMEM_BYTES = RING_BYTES + COLV_BYTES + BAR_BYTES + 1024;  // + alignment
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 54 KB
+constexpr uint32_t LR_A_BYTES = BM * 64 * 2;         // L half: 128 rows x 64 bf16
+constexpr uint32_t LR_B_BYTES = BN * 64 * 2;         // proj_up half: 256 rows x 64 bf16
+static_assert(LR_A_BYTES <= A_BYTES && LR_B_BYTES <= B_BYTES, "low-rank halves fit a slot");
+constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
+constexpr int OUT_COLS = 64;                         // columns per TMA store box
+constexpr uint32_t OUT_WARP_BYTES = 32 * OUT_COLS * 2;   // 32 rows x 128 B
+constexpr uint32_t OUT_BYTES = NUM_EPI_WARPS * OUT_WARP_BYTES;
+constexpr uint32_t COLV_BYTES = 2 * 2 * BN * 4;      // wcscales, bias (fp32), 2 tile buffers
+constexpr uint32_t BAR_BYTES = 128;
+constexpr uint32_t SMEM_BYTES = RING_BYTES + OUT_BYTES + COLV_BYTES + BAR_BYTES + 1024;
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0;
 constexpr uint32_t TM_LR = 256;
-constexpr uint32_t TM_SFA = 256;
-constexpr uint32_t TM_SFB = 272;
+constexpr uint32_t TM_SF = 256;                      // per slot: 16 SFA + 32 SFB columns
+constexpr uint32_t TM_SF_SLOT = 48;
+static_assert(TM_SF + STAGES * TM_SF_SLOT <= TMEM_COLS, "scale columns fit");
+static_assert(STAGE_BYTES % 1024 == 0, "slots and the output buffers stay 1024-aligned");
 
 // Wait-site ids recorded in the error word.
 constexpr uint32_t SITE_PROD = 0x10, SITE_MMA_TE = 0x11, SITE_MMA_FULL = 0x12,
@@ -76,8 +84,7 @@ struct Params {
   const __nv_bfloat16* wcscales;
   const __nv_bfloat16* wtscale;
   const __nv_bfloat16* bias;  // may be null
-  __nv_bfloat16* y;
-  int M, N, K, ldy;
+  int M, N, K;
   int m_tiles, n_tiles;
 };
 
@@ -86,29 +93,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2] u8
-                   const __grid_constant__ CUtensorMap tm_b,   // qweight[N, K/2] u8
-                   const __grid_constant__ CUtensorMap tm_l,   // lowrank[M, 128] bf16
-                   const __grid_constant__ CUtensorMap tm_p,   // proj_up[N, 128] bf16
+w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/2] u8, box {128, 128}
+                   const __grid_constant__ CUtensorMap tm_b,   // qweight [N, K/2] u8, box {128, 256}
+                   const __grid_constant__ CUtensorMap tm_l,   // lowrank [M, 128] bf16, box {64, 128}
+                   const __grid_constant__ CUtensorMap tm_p,   // proj_up [N, 128] bf16, box {64, 256}
+                   const __grid_constant__ CUtensorMap tm_y,   // y [M, ldy] bf16, box {64, 32}
                    const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t s_a = smem_u32(smem);
-  const uint32_t s_b = s_a + STAGES * A_BYTES;
-  const uint32_t s_sfa = s_b + STAGES * B_BYTES;
-  const uint32_t s_sfb = s_sfa + STAGES * SFA_BYTES;
-  const uint32_t s_colv = s_sfb + STAGES * SFB_BYTES;
+  const uint32_t s_ring = smem_u32(smem);
+  auto s_a = [&](uint32_t s) { return s_ring + s * STAGE_BYTES; };
+  auto s_b = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + A_BYTES; };
+  auto s_sfa = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + A_BYTES + B_BYTES; };
+  auto s_sfb = [&](uint32_t s) {
+    return s_ring + s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES;
+  };
+  const uint32_t s_out = s_ring + RING_BYTES;
+  const uint32_t s_colv = s_out + OUT_BYTES;
   const uint32_t s_bar = s_colv + COLV_BYTES;
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
@@ -117,7 +120,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
   const uint32_t drain_bar = tmem_full_bar + 16u;
   const uint32_t final_bar = tmem_full_bar + 24u;
   const uint32_t tmem_slot = tmem_full_bar + 32u;
-  uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_a));
+  uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -127,6 +130,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_l);
     prefetch_tmap(&tm_p);
+    prefetch_tmap(&tm_y);
     for (uint32_t s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
@@ -146,9 +150,9 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
 
-  const int num_k = p.K / BK;
+  const int num_k = p.K / BK;                  // K steps per tile
   const int tiles = p.m_tiles * p.n_tiles;
-  const size_t ka_per_rowtile = static_cast<size_t>(p.K / 64);
+  const size_t kblocks = static_cast<size_t>(p.K / 64);   // 512-byte scale blocks per 128 rows
 
   if (warp == 0) {
     if (lane == 0) {
@@ -158,31 +162,28 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int mb = t % p.m_tiles;
         const int nb = t / p.m_tiles;
-        for (int kb = 0; kb < num_k + 2; ++kb, ++it) {
+        for (int st = 0; st < num_k + 2; ++st, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!svdq_wait(empty_bar(s), ph ^ 1u, SITE_PROD)) {
             ok = false;
             break;
           }
-          if (kb < num_k) {
-            mbar_arrive_expect_tx(full_bar(s), STAGE_TX);
-            tma_load_2d(s_a + s * A_BYTES, &tm_a, kb * BK_BYTES, mb * BM, full_bar(s));
-            tma_load_2d(s_b + s * B_BYTES, &tm_b, kb * BK_BYTES, nb * BN, full_bar(s));
-            const uint8_t* sfa_src =
-                p.ascales_tiled + (static_cast<size_t>(mb) * ka_per_rowtile + kb * 4) * 512;
-            const uint8_t* sfb_src0 =
-                p.wscales_tiled + (static_cast<size_t>(2 * nb) * ka_per_rowtile + kb * 4) * 512;
-            const uint8_t* sfb_src1 =
-                p.wscales_tiled + (static_cast<size_t>(2 * nb + 1) * ka_per_rowtile + kb * 4) * 512;
-            bulk_load(s_sfa + s * SFA_BYTES, sfa_src, SFA_BYTES, full_bar(s));
-            bulk_load(s_sfb + s * SFB_BYTES, sfb_src0, SFB_BYTES / 2, full_bar(s));
-            bulk_load(s_sfb + s * SFB_BYTES + SFB_BYTES / 2, sfb_src1, SFB_BYTES / 2, full_bar(s));
+          if (st < num_k) {
+            mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+            tma_load_2d(s_a(s), &tm_a, st * BK_BYTES, mb * BM, full_bar(s));
+            tma_load_2d(s_b(s), &tm_b, st * BK_BYTES, nb * BN, full_bar(s));
+            bulk_load(s_sfa(s),
+                      p.ascales_tiled + (static_cast<size_t>(mb) * kblocks + 4 * st) * 512,
+                      SFA_BYTES, full_bar(s));
+            bulk_load(s_sfb(s),
+                      p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * st) * 1024,
+                      SFB_BYTES, full_bar(s));
           } else {
-            const int j = kb - num_k;  // low-rank K half: r in [64 j, 64 j + 64)
-            mbar_arrive_expect_tx(full_bar(s), LR_TX);
-            tma_load_2d(s_a + s * A_BYTES, &tm_l, j * 64, mb * BM, full_bar(s));
-            tma_load_2d(s_b + s * B_BYTES, &tm_p, j * 64, nb * BN, full_bar(s));
+            const int hr = st - num_k;           // which 64-wide half of R
+            mbar_arrive_expect_tx(full_bar(s), LR_A_BYTES + LR_B_BYTES);
+            tma_load_2d(s_a(s), &tm_l, hr * 64, mb * BM, full_bar(s));
+            tma_load_2d(s_b(s), &tm_p, hr * 64, nb * BN, full_bar(s));
           }
         }
       }
@@ -205,7 +206,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
         if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_MMA_TE)) break;
         tc_fence_after();
-        for (int kb = 0; kb < num_k; ++kb, ++it) {
+        for (int st = 0; st < num_k; ++st, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
@@ -213,27 +214,27 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = s_a + s * A_BYTES;
-          const uint32_t b0 = s_b + s * B_BYTES;
-          const uint32_t sfa0 = s_sfa + s * SFA_BYTES;
-          const uint32_t sfb0 = s_sfb + s * SFB_BYTES;
+          // Scale blocks of this K step: 4 for A (one per 128 rows x 64 k),
+          // 4 x 2 halves for B, each into its own TMEM columns of the slot.
+          const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
+          const uint32_t sfb_t = sfa_t + 16;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            tmem_cp_32x128b_warpx4(tmem_base + TM_SFA + 4 * j,
-                                   smem_desc(sfa0 + 512 * j, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4(sfa_t + 4 * j,
+                                   smem_desc(s_sfa(s) + 512 * j, 0, 128, kLayoutSwizzleNone));
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
+          for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int h = 0; h < 2; ++h)
               tmem_cp_32x128b_warpx4(
-                  tmem_base + TM_SFB + 8 * j + 4 * h,
-                  smem_desc(sfb0 + (SFB_BYTES / 2) * h + 512 * j, 0, 128, kLayoutSwizzleNone));
+                  sfb_t + 8 * j + 4 * h,
+                  smem_desc(s_sfb(s) + 1024 * j + 512 * h, 0, 128, kLayoutSwizzleNone));
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            mma_nvfp4(tmem_base + TM_ACC, smem_desc(a0 + 32 * j, 16, 1024, kLayoutSwizzle128B),
-                      smem_desc(b0 + 32 * j, 16, 1024, kLayoutSwizzle128B), idesc_main,
-                      tmem_base + TM_SFA + 4 * j, tmem_base + TM_SFB + 8 * j,
-                      (kb | j) != 0 ? 1u : 0u);
+            mma_nvfp4(tmem_base + TM_ACC,
+                      smem_desc(s_a(s) + 32 * j, 16, 1024, kLayoutSwizzle128B),
+                      smem_desc(s_b(s) + 32 * j, 16, 1024, kLayoutSwizzle128B), idesc_main,
+                      sfa_t + 4 * j, sfb_t + 8 * j, (st | j) != 0 ? 1u : 0u);
           }
           tc_commit(empty_bar(s));
         }
@@ -243,7 +244,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
         tc_commit(drain_bar);
         if (!svdq_wait(drain_bar, tc & 1u, SITE_MMA_DRAIN)) break;
         tc_fence_after();
-        for (int j = 0; j < 2; ++j, ++it) {
+        for (int hr = 0; hr < 2 && ok; ++hr, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
@@ -251,14 +252,12 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = s_a + s * A_BYTES;
-          const uint32_t b0 = s_b + s * B_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_f16(tmem_base + TM_LR, smem_desc(a0 + 32 * kk, 16, 1024, kLayoutSwizzle128B),
-                    smem_desc(b0 + 32 * kk, 16, 1024, kLayoutSwizzle128B), idesc_lr,
-                    (j | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem_base + TM_LR,
+                    smem_desc(s_a(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B),
+                    smem_desc(s_b(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B), idesc_lr,
+                    (hr | kk) != 0 ? 1u : 0u);
           tc_commit(empty_bar(s));
         }
         if (!ok) break;
@@ -275,8 +274,10 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
     const int et = threadIdx.x - 64;     // 0..255
     const float alpha = __bfloat162float(p.wtscale[0]);
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    float* colv = reinterpret_cast<float*>(smem + (s_colv - s_a));
+    const uint32_t s_obuf = s_out + static_cast<uint32_t>(warp - 2) * OUT_WARP_BYTES;
+    float* colv = reinterpret_cast<float*>(smem + (s_colv - s_ring));
     uint32_t tc = 0;
+    bool ok = true;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int mb = t % p.m_tiles;
       const int nb = t / p.m_tiles;
@@ -294,11 +295,13 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
         wc_s[et] = wcv * alpha;
         bs_s[et] = bsv;
       }
+      // Every epilogue warp passes this barrier once per tile, also after a
+      // failed wait, so that no warp is left waiting on it.
       named_bar_sync(2, 32 * NUM_EPI_WARPS);
-      if (!__all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI))) break;
+      if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI));
+      if (!ok) continue;
       tc_fence_after();
-      const int row = mb * BM + q * 32 + lane;
-      uint32_t out[4][16];
+      uint32_t out[8][8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const int col = half * 128 + 16 * c;
@@ -314,28 +317,38 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact   [M, K/2
                                 __uint_as_float(lr[2 * i]) + b2.x);
           const float o1 = fmaf(__uint_as_float(acc[2 * i + 1]), w2.y,
                                 __uint_as_float(lr[2 * i + 1]) + b2.y);
-          out[c >> 1][8 * (c & 1) + i] = pack_bf16x2(o0, o1);
+          out[c][i] = pack_bf16x2(o0, o1);
         }
       }
       // TMEM is free for the next tile as soon as every warp has its values.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tmem_empty_bar);
-      if (row < p.M) {
-        __nv_bfloat16* yrow = p.y + static_cast<size_t>(row) * p.ldy;
+      // Rows -> swizzled buffer (row = lane, 128 B per row; 16-byte chunk
+      // j of row r at chunk j ^ (r % 8), the TMA 128-byte swizzle) -> TMA
+      // store of 32 rows x 64 columns, twice per tile.
+      const int row0 = mb * BM + q * 32;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int n0 = nb * BN + half * 128 + 32 * c;
-          if (n0 < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+      for (int pc = 0; pc < 2; ++pc) {
+        if (lane == 0) bulk_wait_group_read0();   // previous store has read the buffer
+        __syncwarp();
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(out[c][4 * v], out[c][4 * v + 1], out[c][4 * v + 2],
-                                  out[c][4 * v + 3]);
-          }
+        for (int j = 0; j < 8; ++j) {
+          const int c = 4 * pc + (j >> 1);
+          const int v = j & 1;
+          st_shared_v4(s_obuf + lane * 128 + ((j ^ (lane & 7)) << 4), out[c][4 * v],
+                       out[c][4 * v + 1], out[c][4 * v + 2], out[c][4 * v + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int x0 = nb * BN + half * 128 + pc * OUT_COLS;
+        if (lane == 0 && x0 < p.N && row0 < p.M) {
+          tma_store_2d(&tm_y, s_obuf, x0, row0);
+          bulk_commit_group();
         }
       }
     }
+    if (lane == 0) bulk_wait_group0();
   }
 
   // ----------------------------------------------------------- teardown --

@@ -23,11 +23,11 @@
 // ulp), so the conversion sees the tie.  A scale that rounds to zero gives
 // r = 0 and therefore signed zero codes.
 //
-// CTA layout: a tile of BM rows (32..128) over a K range, 18 warps.
-//   warp 0      TMA producer: per stage of 128 k, the x tile as two
+// CTA layout: a tile of BM rows (32..256) over a K range, 18 warps.
+//   warp 0      TMA producer: per stage of 64 or 128 k, the x tile as
 //               [BM rows x 64 k] bf16 boxes (128-byte swizzle), proj_down
-//               rows [128 k x 128 r] (four 64 x 64 boxes) and the 128 smooth
-//               values, into a ring of stages.
+//               rows [64 k x 128 r] per box pair (64 x 64 boxes) and the
+//               smooth values, into a ring of stages.
 //   warp 1      TMEM owner, MMA issuer.  The low-rank product is computed
 //               transposed, L^T[128 x BM] += proj_down_chunk^T x_tile^T:
 //               tcgen05.mma kind::f16, M = 128 (= R), N = BM, K = 16;
@@ -54,14 +54,11 @@ namespace kq {
 
 constexpr int R = 128;                 // rank (MMA M)
 constexpr int BKE = 64;                // k per chunk (one 128-byte swizzled box row)
-constexpr int CPS = 2;                 // chunks per stage
-constexpr int MAX_BM = 128;
+constexpr int MAX_BM = 256;
 constexpr int MAX_STAGES = 6;
 constexpr uint32_t PD_BOX = 64 * 64 * 2;          // [64 k x 64 r] bf16 box, 8 KB
 constexpr uint32_t PD_CHUNK = 2 * PD_BOX;         // one chunk of proj_down, 16 KB
-constexpr uint32_t PD_BYTES = CPS * PD_CHUNK;     // 32 KB per stage
 constexpr uint32_t SMOOTH_CHUNK = BKE * 2;        // 128 B
-constexpr uint32_t SMOOTH_BYTES = CPS * SMOOTH_CHUNK;
 constexpr int NUM_QWARPS = 16;
 constexpr int NUM_QTHREADS = NUM_QWARPS * 32;
 constexpr int NUM_THREADS = 64 + NUM_QTHREADS;
@@ -71,24 +68,35 @@ constexpr int PART_STRIDE = R + 4;  // floats per row m of the partial-L buffer
 
 constexpr uint32_t SITE_PROD = 0x20, SITE_MMA = 0x21, SITE_QUANT = 0x22, SITE_LFULL = 0x23;
 
+// A stage holds `cps` chunks of 64 k (1 or 2): x [bm rows x 128 B] per
+// chunk, proj_down [64 k x 128 r] per chunk, 128 B of smooth per chunk.
 __host__ __device__ constexpr uint32_t x_chunk(int bm) { return static_cast<uint32_t>(bm) * 128u; }
-__host__ __device__ constexpr uint32_t x_bytes(int bm) { return CPS * x_chunk(bm); }
-__host__ __device__ constexpr uint32_t stage_bytes(int bm) {
-  return (x_bytes(bm) + PD_BYTES + SMOOTH_BYTES + 1023u) & ~1023u;
+__host__ __device__ constexpr uint32_t x_bytes(int bm, int cps) { return cps * x_chunk(bm); }
+__host__ __device__ constexpr uint32_t stage_bytes(int bm, int cps) {
+  return (cps * (x_chunk(bm) + PD_CHUNK + SMOOTH_CHUNK) + 1023u) & ~1023u;
 }
-__host__ __device__ constexpr int num_stages(int bm) {
-  return (SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm) < MAX_STAGES
-             ? static_cast<int>((SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm))
+__host__ __device__ constexpr int num_stages(int bm, int cps) {
+  return (SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm, cps) < MAX_STAGES
+             ? static_cast<int>((SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm, cps))
              : MAX_STAGES;
 }
-__host__ __device__ constexpr uint32_t smem_bytes(int bm) {
-  return num_stages(bm) * stage_bytes(bm) + BAR_BYTES + 1024;
+__host__ __device__ constexpr uint32_t smem_bytes(int bm, int cps) {
+  return num_stages(bm, cps) * stage_bytes(bm, cps) + BAR_BYTES + 1024;
+}
+// Two chunks per stage when that still leaves three stages in flight.
+__host__ __device__ constexpr int chunks_per_stage(int bm) {
+  return num_stages(bm, 2) >= 3 ? 2 : 1;
 }
 __host__ __device__ constexpr uint32_t tmem_cols(int bm) {
-  return bm <= 32 ? 32u : bm <= 64 ? 64u : 128u;
+  return bm <= 32 ? 32u : bm <= 64 ? 64u : bm <= 128 ? 128u : 256u;
 }
-static_assert(MAX_BM * PART_STRIDE * 4 <= 2 * stage_bytes(MAX_BM), "partial buffer fits the ring");
-static_assert(num_stages(32) >= 2 && num_stages(MAX_BM) >= 2, "at least two stages");
+static_assert(MAX_BM * PART_STRIDE * 4 <=
+                  num_stages(MAX_BM, chunks_per_stage(MAX_BM)) *
+                      stage_bytes(MAX_BM, chunks_per_stage(MAX_BM)),
+              "partial buffer fits the ring");
+static_assert(num_stages(32, chunks_per_stage(32)) >= 3 &&
+                  num_stages(MAX_BM, chunks_per_stage(MAX_BM)) >= 3,
+              "at least three stages");
 
 struct Params {
   const __nv_bfloat16* smooth;
@@ -98,7 +106,7 @@ struct Params {
   int M, K;
   int chunks;  // K / 64
   int split;   // CTAs per cluster along K
-  int bm;      // rows per CTA (multiple of 32, <= 128)
+  int bm;      // rows per CTA (multiple of 32, <= 256)
 };
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
@@ -197,16 +205,19 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int bm = p.bm;
-  const uint32_t sbytes = stage_bytes(bm);
-  const uint32_t nst = static_cast<uint32_t>(num_stages(bm));
+  const int cps = chunks_per_stage(bm);
+  const uint32_t sbytes = stage_bytes(bm, cps);
+  const uint32_t nst = static_cast<uint32_t>(num_stages(bm, cps));
   const uint32_t s_ring = smem_u32(smem);
   const uint32_t s_bar = s_ring + nst * sbytes;
-  // Stage layout: x chunks [CPS][bm rows x 128 B], proj_down chunks
-  // [CPS][r half][64 k x 128 B], smooth chunks [CPS][128 B].
+  // Stage layout: x chunks [cps][bm rows x 128 B], proj_down chunks
+  // [cps][r half][64 k x 128 B], smooth chunks [cps][128 B].
   auto s_x = [&](uint32_t s, int c) { return s_ring + s * sbytes + c * x_chunk(bm); };
-  auto s_pd = [&](uint32_t s, int c) { return s_ring + s * sbytes + x_bytes(bm) + c * PD_CHUNK; };
+  auto s_pd = [&](uint32_t s, int c) {
+    return s_ring + s * sbytes + x_bytes(bm, cps) + c * PD_CHUNK;
+  };
   auto s_sm = [&](uint32_t s, int c) {
-    return s_ring + s * sbytes + x_bytes(bm) + PD_BYTES + c * SMOOTH_CHUNK;
+    return s_ring + s * sbytes + x_bytes(bm, cps) + cps * PD_CHUNK + c * SMOOTH_CHUNK;
   };
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (MAX_STAGES + s); };
@@ -222,9 +233,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   const int rank = blockIdx.x;  // == rank in the cluster (cluster dims = (split, 1, 1))
   const int c_begin = rank * p.chunks / p.split;
   const int c_end = (rank + 1) * p.chunks / p.split;
-  // >= 1 chunk per CTA (host guarantees split <= chunks); stages of CPS
+  // >= 1 chunk per CTA (host guarantees split <= chunks); stages of cps
   // chunks, the last one possibly partial.
-  const int nstages = (c_end - c_begin + CPS - 1) / CPS;
+  const int nstages = (c_end - c_begin + cps - 1) / cps;
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_x);
@@ -260,8 +271,8 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
           ok = false;
           break;
         }
-        const int kc0 = c_begin + CPS * i;
-        const int nc = c_end - kc0 < CPS ? c_end - kc0 : CPS;
+        const int kc0 = c_begin + cps * i;
+        const int nc = c_end - kc0 < cps ? c_end - kc0 : cps;
         mbar_arrive_expect_tx(full_bar(s), nc * (x_chunk(bm) + PD_CHUNK + SMOOTH_CHUNK));
         for (int c = 0; c < nc; ++c) {
           const int kc = kc0 + c;
@@ -295,8 +306,8 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
           break;
         }
         tc_fence_after();
-        const int kc0 = c_begin + CPS * i;
-        const int nc = c_end - kc0 < CPS ? c_end - kc0 : CPS;
+        const int kc0 = c_begin + cps * i;
+        const int nc = c_end - kc0 < cps ? c_end - kc0 : cps;
         for (int c = 0; c < nc; ++c) {
 #pragma unroll
           for (int kk = 0; kk < BKE / 16; ++kk) {
@@ -324,14 +335,15 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
         ok = false;
         break;
       }
-      const int kc0 = c_begin + CPS * i;
-      const int nc = c_end - kc0 < CPS ? c_end - kc0 : CPS;
-      // bm rows x (4 nc) groups; lanes 8j..8j+7 take one row's 8 groups
-      // (chunk c = lane / 4 % 2, group g = lane % 4), whole warps together.
-      for (int gi = qt; gi < bm * 4 * CPS; gi += NUM_QTHREADS) {
-        const int r = gi >> 3;       // row in the tile
-        const int c = (gi >> 2) & 1; // chunk within the stage
-        const int g = gi & 3;        // group of 16 within the chunk
+      const int kc0 = c_begin + cps * i;
+      const int nc = c_end - kc0 < cps ? c_end - kc0 : cps;
+      // bm rows x (4 cps) groups; consecutive lanes take one row's groups
+      // (chunk c, then group g of 16 within it), whole warps together.
+      const int gshift = cps == 2 ? 3 : 2;   // log2(groups per row per stage)
+      for (int gi = qt; gi < (bm << gshift); gi += NUM_QTHREADS) {
+        const int r = gi >> gshift;               // row in the tile
+        const int c = (gi >> 2) & (cps - 1);      // chunk within the stage
+        const int g = gi & 3;                     // group of 16 within the chunk
         const bool active = c < nc;     // the stage's second chunk may be absent
         const int row = mb * bm + r;
         const int kc = kc0 + c;

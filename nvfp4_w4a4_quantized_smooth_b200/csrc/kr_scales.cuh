@@ -1,14 +1,16 @@
 // kr_scales.cuh -- scale-factor tile order, and two small elementwise
 // kernels (scale unpack for tests, SiLU * mul for the feed-forward block).
 //
-// Tile order of every scale buffer the GEMM reads (activation scales and
-// weight scales alike): rows are cut into tiles of 128, K into blocks of
-// 64 (4 scales of 16).  Each (row tile t, K block b) pair is one 512-byte
-// block at offset (t * (K/64) + b) * 512, holding scale (row, 4 b + j) at
-// byte (row % 32) * 16 + ((row % 128) / 32) * 4 + j.  That is the layout
-// tcgen05.cp (32x128b, warpx4) turns into the TMEM scale-factor layout of
-// tcgen05.mma kind::mxf4nvf4: TMEM lane row % 32 (in every lane quarter),
-// column (row % 128) / 32, byte j.
+// Tile order of the activation scales: rows are cut into tiles of 128, K
+// into blocks of 64 (4 scales of 16).  Each (row tile t, K block b) pair is
+// one 512-byte block at offset (t * (K/64) + b) * 512, holding scale
+// (row, 4 b + j) at byte (row % 32) * 16 + ((row % 128) / 32) * 4 + j.
+// That is the layout tcgen05.cp (32x128b, warpx4) turns into the TMEM
+// scale-factor layout of tcgen05.mma kind::mxf4nvf4: TMEM lane row % 32 (in
+// every lane quarter), column (row % 128) / 32, byte j.
+// The weight scales use the same 512-byte blocks, ordered for 256-row GEMM
+// tiles: block ((T * (K/64) + b) * 2 + h) holds rows 256 T + 128 h + [0, 128)
+// of K block b, so one tile's scales over a run of K are contiguous.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -22,11 +24,17 @@ __device__ __forceinline__ size_t tiled_offset(int row, int kg, int kblocks) {
   return (static_cast<size_t>(t) * kblocks + b) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4 + j;
 }
 
+__device__ __forceinline__ size_t weight_tiled_offset(int row, int kg, int kblocks) {
+  const int T = row >> 8, h = (row >> 7) & 1, b = kg >> 2, j = kg & 3;
+  return ((static_cast<size_t>(T) * kblocks + b) * 2 + h) * 512 + (row & 31) * 16 +
+         ((row & 127) >> 5) * 4 + j;
+}
+
 // Device counter of rejected scale bytes (sign bit set, or NaN 0x7F).
 __device__ uint32_t g_bad_scales = 0;
 
-// wscales [K/16, N] (N contiguous) -> tiled, rows padded to `rows_pad`
-// with zero scales.  One thread per output word (4 scales of one row).
+// wscales [K/16, N] (N contiguous) -> weight tile order, rows padded to
+// `rows_pad` (a multiple of 256) with zero scales.  One thread per output word (4 scales of one row).
 __global__ void repack_weight_scales_kernel(const uint8_t* __restrict__ ws, int N, int K,
                                             int rows_pad, uint8_t* __restrict__ out) {
   const int kblocks = K / 64;
@@ -38,9 +46,10 @@ __global__ void repack_weight_scales_kernel(const uint8_t* __restrict__ ws, int 
     // word inside the 512-byte block.
     const size_t blk = w >> 7;
     const int wi = static_cast<int>(w & 127);
-    const int t = static_cast<int>(blk / kblocks);
-    const int b = static_cast<int>(blk % kblocks);
-    const int row = t * 128 + ((wi & 3) << 5) + (wi >> 2);
+    const int h = static_cast<int>(blk & 1);
+    const int T = static_cast<int>((blk >> 1) / kblocks);
+    const int b = static_cast<int>((blk >> 1) % kblocks);
+    const int row = T * 256 + h * 128 + ((wi & 3) << 5) + (wi >> 2);
     uint32_t word = 0;
     if (row < N) {
 #pragma unroll
@@ -55,16 +64,18 @@ __global__ void repack_weight_scales_kernel(const uint8_t* __restrict__ ws, int 
   if (bad) atomicAdd(&g_bad_scales, bad);
 }
 
-// tiled -> [rows, K/16] (row-major), the logical scale matrix.
+// tiled (activation or weight order) -> [rows, K/16] (row-major), the
+// logical scale matrix.
 __global__ void unpack_scales_kernel(const uint8_t* __restrict__ tiled, int rows, int K,
-                                     uint8_t* __restrict__ out) {
+                                     int weight_order, uint8_t* __restrict__ out) {
   const int kg_n = K / 16;
   const size_t total = static_cast<size_t>(rows) * kg_n;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int row = static_cast<int>(i / kg_n);
     const int kg = static_cast<int>(i % kg_n);
-    out[i] = tiled[tiled_offset(row, kg, K / 64)];
+    out[i] = tiled[weight_order ? weight_tiled_offset(row, kg, K / 64)
+                                : tiled_offset(row, kg, K / 64)];
   }
 }
 

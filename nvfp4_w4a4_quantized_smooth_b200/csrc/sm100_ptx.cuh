@@ -70,6 +70,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0u;
 }
 
+// Same test, but the thread may sleep in hardware for up to `hint_ns`
+// until the phase completes, instead of spinning on the issue slots that
+// the working warps of the SM need.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0u;
+}
+
 // Bounded wait for the phase with the given parity to complete.  Returns
 // false if the limit ran out (the error word is then set) or if another
 // thread already raised an error.  `site` identifies the wait.
@@ -77,14 +93,12 @@ __device__ __forceinline__ bool svdq_wait(uint32_t bar, uint32_t parity, uint32_
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   const uint64_t limit = *(volatile uint64_t*)&g_wait_limit_ns;
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 31u) == 0u) {
-      if (error_raised()) return false;
-      if (globaltimer_ns() - t0 > limit) {
-        raise_timeout(site);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (error_raised()) return false;
+    if (globaltimer_ns() - t0 > limit) {
+      raise_timeout(site);
+      return false;
     }
   }
 }
@@ -112,6 +126,45 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int3
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// 3-D tiled bulk tensor load global -> shared (this CTA), completion on bar.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                            int32_t z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// 2-D tiled bulk tensor store shared (this CTA) -> global, tracked by the
+// issuing thread's bulk async-group.  Elements outside the tensor map's
+// extent are not written.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed store of this thread has finished READING its
+// shared-memory source (the buffer may then be rewritten).
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+// Wait until every committed store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Contiguous bulk copy global -> shared; 16-byte aligned, size % 16 == 0.
@@ -259,6 +312,7 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(uint32_t M, uint32_t N) {
          | (0u << 23)               // scale format: ue4m3
          | ((M >> 4) << 24);        // M / 16
 }
+
 
 // --------------------------------------------------------------- cluster --
 __device__ __forceinline__ uint32_t cluster_ctarank() {

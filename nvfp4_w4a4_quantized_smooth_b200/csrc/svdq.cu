@@ -25,7 +25,7 @@ struct DeviceInfo {
   int num_sms = 0;
   // Max co-resident clusters of the activation kernel, by (bm / 32, split);
   // -1 = not queried yet.
-  int kq_clusters[9][9];
+  int kq_clusters[9][9];   // [bm / 32][split]
 };
 
 std::mutex g_mu;
@@ -79,15 +79,16 @@ int device_setup(DeviceInfo** out) {
 
 // 2-D tensor map over a row-major matrix: `inner` contiguous elements per
 // row (row pitch `pitch_bytes`), `outer` rows; box `box_inner` x
-// `box_outer`, 128-byte swizzle, zero fill outside the matrix.
+// `box_outer`, 128-byte swizzle (or none), zero fill outside the matrix.
 int make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
-              uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {pitch_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
@@ -116,7 +117,7 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(split, 1024, 1);
   cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = svdq::kq::smem_bytes(bm);
+  cfg.dynamicSmemBytes = svdq::kq::smem_bytes(bm, svdq::kq::chunks_per_stage(bm));
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = split;
@@ -134,31 +135,30 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
   return n;
 }
 
-// Row tile and K split of the activation kernel: the single-wave grid
-// (m_tiles clusters of `split` CTAs, at most one CTA per SM, every cluster
-// co-resident) that occupies the most SMs; ties go to less row padding, then
-// to the larger row tile (less proj_down traffic per row).
+// Row tile and K split of the activation kernel: among the grids that run
+// in one wave (m_tiles clusters of `split` CTAs, split a power of two, at
+// most one CTA per SM, every cluster co-resident), the one that occupies
+// the most SMs; ties go to the smaller split (less partial-sum traffic),
+// then to the larger row tile (less proj_down traffic per row).  If none
+// fits (very large M), the largest tile without a split.
 void kq_plan(DeviceInfo* d, int M, int chunks, int* bm_out, int* split_out) {
-  int best_bm = svdq::kq::MAX_BM, best_split = 1, best_score = -1, best_waste = 0;
+  int best_bm = svdq::kq::MAX_BM, best_split = 1, best_ctas = -1;
   for (int bm = svdq::kq::MAX_BM; bm >= 32; bm -= 32) {
     const int m_tiles = (M + bm - 1) / bm;
-    const int waste = m_tiles * bm - M;
-    for (int split = 1; split <= 8 && split <= chunks; ++split) {
+    for (int split = 1; split <= 8 && split <= chunks; split *= 2) {
       const int ctas = m_tiles * split;
       if (ctas > d->num_sms) break;
       if (m_tiles > kq_max_clusters(d, bm, split)) continue;
-      if (ctas > best_score || (ctas == best_score && waste < best_waste)) {
-        best_score = ctas;
-        best_waste = waste;
+      if (ctas > best_ctas || (ctas == best_ctas && split < best_split)) {
+        best_ctas = ctas;
         best_bm = bm;
         best_split = split;
       }
     }
   }
-  *bm_out = best_bm;        // no single-wave plan: largest tile, no split
+  *bm_out = best_bm;
   *split_out = best_split;
 }
-
 }  // namespace
 
 extern "C" {
@@ -258,7 +258,7 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(split, m_tiles, 1);
   cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = svdq::kq::smem_bytes(bm);
+  cfg.dynamicSmemBytes = svdq::kq::smem_bytes(bm, svdq::kq::chunks_per_stage(bm));
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -289,8 +289,8 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   DeviceInfo* d = nullptr;
   if (int st = device_setup(&d)) return st;
 
-  CUtensorMap tm_a, tm_b, tm_l, tm_p;
   const uint64_t kb = static_cast<uint64_t>(K) / 2;
+  CUtensorMap tm_a, tm_b, tm_l, tm_p, tm_y;
   if (make_tmap(&tm_a, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, svdq::kg::BK_BYTES,
                 svdq::kg::BM) ||
       make_tmap(&tm_b, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, N, kb, svdq::kg::BK_BYTES,
@@ -298,7 +298,9 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
       make_tmap(&tm_l, lowrank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, M,
                 static_cast<uint64_t>(R) * 2, 64, svdq::kg::BM) ||
       make_tmap(&tm_p, proj_up, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, N,
-                static_cast<uint64_t>(R) * 2, 64, svdq::kg::BN))
+                static_cast<uint64_t>(R) * 2, 64, svdq::kg::BN) ||
+      make_tmap(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(ldy) * 2,
+                svdq::kg::OUT_COLS, 32))
     return SVDQ_ERR_CUDA;
 
   svdq::kg::Params p;
@@ -307,17 +309,16 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   p.wcscales = reinterpret_cast<const __nv_bfloat16*>(wcscales);
   p.wtscale = reinterpret_cast<const __nv_bfloat16*>(wtscale);
   p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
-  p.y = reinterpret_cast<__nv_bfloat16*>(y);
   p.M = M;
   p.N = N;
   p.K = K;
-  p.ldy = ldy;
   p.m_tiles = (M + svdq::kg::BM - 1) / svdq::kg::BM;
   p.n_tiles = (N + svdq::kg::BN - 1) / svdq::kg::BN;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < d->num_sms ? tiles : d->num_sms;
   svdq::kg::w4a4_linear_kernel<<<grid, svdq::kg::NUM_THREADS, svdq::kg::SMEM_BYTES,
-                                 static_cast<cudaStream_t>(stream)>>>(tm_a, tm_b, tm_l, tm_p, p);
+                                 static_cast<cudaStream_t>(stream)>>>(tm_a, tm_b, tm_l, tm_p, tm_y,
+                                                                      p);
   return launch_status();
 }
 
@@ -331,8 +332,10 @@ int svdq_quantize_plan(int M, int K, int* bm, int* split) {
   return SVDQ_OK;
 }
 
-int svdq_unpack_scales(const void* scales_tiled, int rows, int K, uint8_t* out, void* stream) {
+int svdq_unpack_scales(const void* scales_tiled, int rows, int K, int kind, uint8_t* out,
+                       void* stream) {
   if (!scales_tiled || !out) return SVDQ_ERR_INVALID_ARG;
+  if (kind != SVDQ_SCALES_ACT && kind != SVDQ_SCALES_WEIGHT) return SVDQ_ERR_INVALID_ARG;
   if (rows < 1 || K < 16 || K % 16) return SVDQ_ERR_SHAPE;
   if (K % 64) return SVDQ_ERR_UNSUPPORTED;
   DeviceInfo* d = nullptr;
@@ -340,7 +343,8 @@ int svdq_unpack_scales(const void* scales_tiled, int rows, int K, uint8_t* out, 
   const size_t total = static_cast<size_t>(rows) * (K / 16);
   svdq::kr::unpack_scales_kernel<<<grid_for(total, 256, d->num_sms), 256, 0,
                                    static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint8_t*>(scales_tiled), rows, K, out);
+      static_cast<const uint8_t*>(scales_tiled), rows, K, kind == SVDQ_SCALES_WEIGHT ? 1 : 0,
+      out);
   return launch_status();
 }
 

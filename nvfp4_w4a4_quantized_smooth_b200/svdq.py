@@ -28,6 +28,11 @@ SVDQ_ERR_ARCH = 5
 SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
+# Constants of include/svdq.h.
+ABI_VERSION = 2
+SCALES_ACT = 0
+SCALES_WEIGHT = 1
+
 # Every symbol include/svdq.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -42,7 +47,7 @@ SIGNATURES = {
     "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
     "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
     "svdq_quantize_plan": (_I, [_I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
-    "svdq_unpack_scales": (_I, [_P, _I, _I, _P, _P]),
+    "svdq_unpack_scales": (_I, [_P, _I, _I, _I, _P, _P]),
     "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
     "svdq_check_device_error": (_I, [_P]),
     "svdq_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
@@ -59,6 +64,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
+    if lib.svdq_abi_version() != ABI_VERSION:
+        raise ImportError(f"{path} has ABI version {lib.svdq_abi_version()}, this binding "
+                          f"expects {ABI_VERSION}: rebuild it")
     return lib
 
 
@@ -184,10 +192,16 @@ def quantize_plan(M: int, K: int):
     return bm.value, split.value
 
 
-def unpack_scales(scales_tiled: torch.Tensor, rows: int, K: int, stream=None) -> torch.Tensor:
-    """Tiled scales -> logical [rows, K/16] uint8 (test / inspection helper)."""
+def unpack_scales(scales_tiled: torch.Tensor, rows: int, K: int, kind: str = "act",
+                  stream=None) -> torch.Tensor:
+    """Tiled scales -> logical [rows, K/16] uint8 (test / inspection helper).
+
+    kind: "act" for svdq_quantize_act's order, "weight" for
+    svdq_repack_weights' order."""
+    code = {"act": SCALES_ACT, "weight": SCALES_WEIGHT}[kind]
     out = torch.empty(rows, K // 16, dtype=torch.uint8, device=scales_tiled.device)
-    _check(_lib.svdq_unpack_scales(_ptr(scales_tiled), rows, K, _ptr(out), _stream(stream)),
+    _check(_lib.svdq_unpack_scales(_ptr(scales_tiled), rows, K, code, _ptr(out),
+                                   _stream(stream)),
            "svdq_unpack_scales")
     return out
 

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(svdq):
 
 
 def test_abi_version_and_status_strings(svdq):
-    assert svdq.abi_version() == 1
+    assert svdq.abi_version() == 2 == svdq.ABI_VERSION
     for st in range(8):
         s = svdq._lib.svdq_status_string(st).decode()
         assert s.startswith("SVDQ")
@@ -100,6 +100,11 @@ def test_argument_checks_fail_before_any_device_work(svdq):
                                  None) == svdq.SVDQ_ERR_ALIGNMENT
     assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, odd, 16, 64,
                                 256, 128, fake, 64, None) == svdq.SVDQ_ERR_ALIGNMENT
+    # scale unpack: only the two documented tile orders
+    for kind in (-1, 2):
+        assert lib.svdq_unpack_scales(fake, 16, 64, kind, fake, None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_unpack_scales(fake, 0, 64, svdq.SCALES_ACT, fake,
+                                  None) == svdq.SVDQ_ERR_SHAPE
 
 
 def test_device_calls_without_a_gpu_report_an_error(svdq):

@@ -37,12 +37,12 @@ def test_repack_round_trip(N, K):
     ws = torch.randint(0, 0x7F, (K // 16, N), generator=g, dtype=torch.uint8)
     t = s.repack_weights(ws.cuda())
     assert t.numel() == s.wscales_tiled_bytes(N, K)
-    back = s.unpack_scales(t, N, K).cpu()
+    back = s.unpack_scales(t, N, K, kind="weight").cpu()
     assert torch.equal(back, ws.t().contiguous())
     # padding rows (beyond N) of the tiled buffer are zero scales
     rows_pad = (N + 255) // 256 * 256
     if rows_pad > N:
-        full = s.unpack_scales(t, rows_pad, K).cpu()
+        full = s.unpack_scales(t, rows_pad, K, kind="weight").cpu()
         assert torch.all(full[N:] == 0)
 
 
@@ -79,11 +79,11 @@ def test_quantize_plans_fit_one_wave():
     for M in (1, 16, 64, 100, 256, 1024, 4352, 17408):
         for K in (64, 512, 3840, 10240):
             bm, split = s.quantize_plan(M, K)
-            assert bm % 32 == 0 and 32 <= bm <= 128, (M, K, bm)
+            assert bm % 32 == 0 and 32 <= bm <= 256, (M, K, bm)
             assert 1 <= split <= min(8, K // 64), (M, K, split)
             tiles = -(-M // bm)
             if tiles * split > torch.cuda.get_device_properties(0).multi_processor_count:
-                assert split == 1 and bm == 128, (M, K, bm, split)
+                assert split == 1 and bm == 256, (M, K, bm, split)
 
 
 def _golden_rows():
