@@ -16,12 +16,16 @@
 //               the low-rank operands, one 64-wide half of R each (L half
 //               in the A place, proj_up half in the B place), so they are
 //               prefetched like any other step.
-//   warp 1      TMEM owner and MMA issuer (one thread): copies the scale
-//               blocks smem -> TMEM (tcgen05.cp), issues
+//   warp 1      TMEM owner and MMA issuer (one thread): issues
 //               tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64)
 //               into the main accumulator, then tcgen05.mma kind::f16
 //               (bf16, K=16) for L @ proj_up^T into a second accumulator.
-//   warps 2..9  epilogue (two warps per TMEM lane quarter, one per half
+//   warp 2      scale copier (one thread): copies each slot's scale blocks
+//               smem -> TMEM (tcgen05.cp 32x128b.warpx4, 12 per K step)
+//               and signals the MMA issuer through a per-slot barrier.
+//               Issued from their own warp, the copies run alongside the
+//               MMAs instead of between them.
+//   warps 3..10 epilogue (two warps per TMEM lane quarter, one per half
 //               of the 256 columns): stage the tile's wcscales / bias in
 //               shared memory while the MMAs run, then TMEM -> registers
 //               (tcgen05.ld), fp32 acc * wtscale * wcscales + lowrank + bias,
@@ -63,9 +67,10 @@ constexpr int OUT_COLS = 64;                         // columns per TMA store bo
 constexpr uint32_t OUT_WARP_BYTES = 32 * OUT_COLS * 2;   // 32 rows x 128 B
 constexpr uint32_t OUT_BYTES = NUM_EPI_WARPS * OUT_WARP_BYTES;
 constexpr uint32_t COLV_BYTES = 2 * 2 * BN * 4;      // wcscales, bias (fp32), 2 tile buffers
-constexpr uint32_t BAR_BYTES = 128;
+constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BYTES = RING_BYTES + OUT_BYTES + COLV_BYTES + BAR_BYTES + 1024;
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int EPI_WARP0 = 3;
+constexpr int NUM_THREADS = 32 * EPI_WARP0 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0;
 constexpr uint32_t TM_LR = 256;
@@ -76,7 +81,8 @@ static_assert(STAGE_BYTES % 1024 == 0, "slots and the output buffers stay 1024-a
 
 // Wait-site ids recorded in the error word.
 constexpr uint32_t SITE_PROD = 0x10, SITE_MMA_TE = 0x11, SITE_MMA_FULL = 0x12,
-                   SITE_MMA_DRAIN = 0x13, SITE_EPI = 0x14;
+                   SITE_MMA_DRAIN = 0x13, SITE_EPI = 0x14, SITE_MMA_SF = 0x15, SITE_CP_TE = 0x16,
+                   SITE_CP_FULL = 0x17;
 
 struct Params {
   const uint8_t* ascales_tiled;
@@ -115,11 +121,13 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
   const uint32_t s_bar = s_colv + COLV_BYTES;
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
-  const uint32_t tmem_full_bar = s_bar + 16u * STAGES;
+  auto sf_full_bar = [&](uint32_t s) { return s_bar + 8u * (2 * STAGES + s); };
+  const uint32_t tmem_full_bar = s_bar + 24u * STAGES;
   const uint32_t tmem_empty_bar = tmem_full_bar + 8u;
   const uint32_t drain_bar = tmem_full_bar + 16u;
   const uint32_t final_bar = tmem_full_bar + 24u;
-  const uint32_t tmem_slot = tmem_full_bar + 32u;
+  const uint32_t cp_final_bar = tmem_full_bar + 32u;
+  const uint32_t tmem_slot = tmem_full_bar + 40u;
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
 
   const int warp = threadIdx.x >> 5;
@@ -134,11 +142,13 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
     for (uint32_t s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
+      mbar_init(sf_full_bar(s), 1);
     }
     mbar_init(tmem_full_bar, 1);
     mbar_init(tmem_empty_bar, NUM_EPI_WARPS);
     mbar_init(drain_bar, 1);
     mbar_init(final_bar, 1);
+    mbar_init(cp_final_bar, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -213,22 +223,13 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
             ok = false;
             break;
           }
+          if (!svdq_wait(sf_full_bar(s), ph, SITE_MMA_SF)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          // Scale blocks of this K step: 4 for A (one per 128 rows x 64 k),
-          // 4 x 2 halves for B, each into its own TMEM columns of the slot.
           const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
           const uint32_t sfb_t = sfa_t + 16;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tmem_cp_32x128b_warpx4(sfa_t + 4 * j,
-                                   smem_desc(s_sfa(s) + 512 * j, 0, 128, kLayoutSwizzleNone));
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tmem_cp_32x128b_warpx4(
-                  sfb_t + 8 * j + 4 * h,
-                  smem_desc(s_sfb(s) + 1024 * j + 512 * h, 0, 128, kLayoutSwizzleNone));
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             mma_nvfp4(tmem_base + TM_ACC,
@@ -247,7 +248,8 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
         for (int hr = 0; hr < 2 && ok; ++hr, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
+          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL) ||
+              !svdq_wait(sf_full_bar(s), ph, SITE_MMA_SF)) {
             ok = false;
             break;
           }
@@ -267,14 +269,57 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
       tc_commit(final_bar);
       drain_wait(final_bar, 0, 100000000ull);
     }
+  } else if (warp == 2) {
+    if (lane == 0) {
+      // -------------------------------------------------- scale copier --
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
+        // The slots' scale columns overlap the low-rank accumulator: wait
+        // until the epilogue has read the previous tile.
+        if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_CP_TE)) break;
+        tc_fence_after();
+        // Every ring slot use is waited on in order, the low-rank slots
+        // included, and every use completes one phase of its slot's
+        // sf_full barrier: a parity wait is then never two phases ahead.
+        for (int st = 0; st < num_k + 2; ++st, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!svdq_wait(full_bar(s), ph, SITE_CP_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (st < num_k) {
+            // 4 A blocks (128 rows x 64 k each), 4 x 2 halves of B blocks.
+            const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
+            const uint32_t sfb_t = sfa_t + 16;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tmem_cp_32x128b_warpx4(sfa_t + 4 * j,
+                                     smem_desc(s_sfa(s) + 512 * j, 0, 128, kLayoutSwizzleNone));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                tmem_cp_32x128b_warpx4(
+                    sfb_t + 8 * j + 4 * h,
+                    smem_desc(s_sfb(s) + 1024 * j + 512 * h, 0, 128, kLayoutSwizzleNone));
+          }
+          tc_commit(sf_full_bar(s));
+        }
+      }
+      tc_commit(cp_final_bar);
+      drain_wait(cp_final_bar, 0, 100000000ull);
+    }
   } else {
     // -------------------------------------------------------- epilogue --
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;    // which 128 of the tile's 256 columns
-    const int et = threadIdx.x - 64;     // 0..255
+    const int half = (warp - EPI_WARP0) >> 2;    // which 128 of the tile's 256 columns
+    const int et = threadIdx.x - 32 * EPI_WARP0;  // 0..255
     const float alpha = __bfloat162float(p.wtscale[0]);
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t s_obuf = s_out + static_cast<uint32_t>(warp - 2) * OUT_WARP_BYTES;
+    const uint32_t s_obuf = s_out + static_cast<uint32_t>(warp - EPI_WARP0) * OUT_WARP_BYTES;
     float* colv = reinterpret_cast<float*>(smem + (s_colv - s_ring));
     uint32_t tc = 0;
     bool ok = true;
