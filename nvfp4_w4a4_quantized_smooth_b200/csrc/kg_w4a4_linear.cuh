@@ -8,24 +8,26 @@
 // with L = x @ proj_down from the activation kernel, stored bf16.
 //
 // Design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer.  A ring of STAGES slots; a slot holds one K
-//               step of 256: the qact box (128 rows x 128 B, 128-byte
-//               swizzle), the qweight box (256 rows x 128 B) and one
-//               contiguous bulk copy each of the step's A and B scale
-//               blocks.  After the K steps of a tile, two more slots carry
-//               the low-rank operands, one 64-wide half of R each (L half
-//               in the A place, proj_up half in the B place), so they are
-//               prefetched like any other step.
-//   warp 1      TMEM owner and MMA issuer (one thread): issues
-//               tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64)
-//               into the main accumulator, then tcgen05.mma kind::f16
-//               (bf16, K=16) for L @ proj_up^T into a second accumulator.
-//   warp 2      scale copier (one thread): copies each slot's scale blocks
-//               smem -> TMEM (tcgen05.cp 32x128b.warpx4, 12 per K step)
-//               and signals the MMA issuer through a per-slot barrier.
-//               Issued from their own warp, the copies run alongside the
-//               MMAs instead of between them.
-//   warps 3..10 epilogue (two warps per TMEM lane quarter, one per half
+//   warp 0      operand producer (one thread).  A ring of AB_SLOTS slots; a
+//               slot holds one K step of 256: the qact box (128 rows x 128 B,
+//               128-byte swizzle) and the qweight box (256 rows x 128 B).
+//               After the K steps of a tile two more slots carry the
+//               low-rank operands, one 64-wide half of R each (L half in the
+//               A place, proj_up half in the B place).
+//   warp 1      TMEM owner and MMA issuer (one thread):
+//               tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64) into
+//               the main accumulator, then tcgen05.mma kind::f16 (bf16,
+//               K=16) for L @ proj_up^T into a second accumulator.
+//   warps 2, 3  scale-factor pipeline: a deeper ring of SF_SLOTS slots, each
+//               one K step's A and B scale blocks (two contiguous bulk
+//               copies, 6 KB), paired with SF_SLOTS TMEM slots.  Warp 3
+//               (one thread) loads a slot as soon as the MMAs that used it
+//               have completed; warp 2 (one thread) copies each loaded slot
+//               smem -> TMEM (tcgen05.cp 32x128b.warpx4, 12 per step).  So
+//               the copies of a step are issued several steps before its
+//               MMAs and never wait on an MMA; issued from their own warp
+//               they run alongside the MMAs.
+//   warps 4..11 epilogue (two warps per TMEM lane quarter, one per half
 //               of the 256 columns): stage the tile's wcscales / bias in
 //               shared memory while the MMAs run, then TMEM -> registers
 //               (tcgen05.ld), fp32 acc * wtscale * wcscales + lowrank + bias,
@@ -34,9 +36,10 @@
 //               swizzled shared-memory buffer to TMA tensor stores, which
 //               write whole rows asynchronously and clip the M / N edges.
 // TMEM map (512 columns, fp32): main accumulator [0, 256), low-rank
-// accumulator [256, 512); the scale factors of the ring slots live in
-// [256, 400) while the main K loop runs (the low-rank MMAs start only after
-// every main MMA has completed).
+// accumulator [256, 512); the scale-factor slots live in [256, 496) while
+// the main K loop runs (the low-rank MMAs start only after every main MMA
+// has completed, and no scale copy of the next tile starts before the
+// epilogue has read this one).
 #pragma once
 
 #include <cuda.h>
@@ -52,37 +55,42 @@ constexpr int BM = 128;          // output rows per tile (MMA M)
 constexpr int BN = 256;          // output columns per tile (MMA N)
 constexpr int BK_BYTES = 128;    // K step: 256 FP4 values = 128 bytes per row
 constexpr int BK = 256;
-constexpr int STAGES = 3;
+constexpr int AB_SLOTS = 3;
+constexpr int SF_SLOTS = 5;
 constexpr uint32_t A_BYTES = BM * BK_BYTES;          // 16 KB
 constexpr uint32_t B_BYTES = BN * BK_BYTES;          // 32 KB
+constexpr uint32_t AB_SLOT_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t SFA_BYTES = 4 * 512;              // 128 rows x 16 scales
 constexpr uint32_t SFB_BYTES = 2 * 4 * 512;          // 256 rows x 16 scales
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 54 KB
+constexpr uint32_t SF_SLOT_BYTES = SFA_BYTES + SFB_BYTES;
 constexpr uint32_t LR_A_BYTES = BM * 64 * 2;         // L half: 128 rows x 64 bf16
 constexpr uint32_t LR_B_BYTES = BN * 64 * 2;         // proj_up half: 256 rows x 64 bf16
 static_assert(LR_A_BYTES <= A_BYTES && LR_B_BYTES <= B_BYTES, "low-rank halves fit a slot");
-constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES;
+constexpr uint32_t AB_RING_BYTES = AB_SLOTS * AB_SLOT_BYTES;
+constexpr uint32_t SF_RING_BYTES = SF_SLOTS * SF_SLOT_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int OUT_COLS = 64;                         // columns per TMA store box
 constexpr uint32_t OUT_WARP_BYTES = 32 * OUT_COLS * 2;   // 32 rows x 128 B
 constexpr uint32_t OUT_BYTES = NUM_EPI_WARPS * OUT_WARP_BYTES;
 constexpr uint32_t COLV_BYTES = 2 * 2 * BN * 4;      // wcscales, bias (fp32), 2 tile buffers
 constexpr uint32_t BAR_BYTES = 256;
-constexpr uint32_t SMEM_BYTES = RING_BYTES + OUT_BYTES + COLV_BYTES + BAR_BYTES + 1024;
-constexpr int EPI_WARP0 = 3;
+constexpr uint32_t SMEM_BYTES =
+    AB_RING_BYTES + SF_RING_BYTES + OUT_BYTES + COLV_BYTES + BAR_BYTES + 1024;
+constexpr int EPI_WARP0 = 4;
 constexpr int NUM_THREADS = 32 * EPI_WARP0 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0;
 constexpr uint32_t TM_LR = 256;
 constexpr uint32_t TM_SF = 256;                      // per slot: 16 SFA + 32 SFB columns
 constexpr uint32_t TM_SF_SLOT = 48;
-static_assert(TM_SF + STAGES * TM_SF_SLOT <= TMEM_COLS, "scale columns fit");
-static_assert(STAGE_BYTES % 1024 == 0, "slots and the output buffers stay 1024-aligned");
+static_assert(TM_SF + SF_SLOTS * TM_SF_SLOT <= TMEM_COLS, "scale columns fit");
+static_assert(AB_SLOT_BYTES % 1024 == 0 && (AB_RING_BYTES + SF_RING_BYTES) % 1024 == 0,
+              "operand slots and the output buffers stay 1024-aligned");
 
 // Wait-site ids recorded in the error word.
 constexpr uint32_t SITE_PROD = 0x10, SITE_MMA_TE = 0x11, SITE_MMA_FULL = 0x12,
-                   SITE_MMA_DRAIN = 0x13, SITE_EPI = 0x14, SITE_MMA_SF = 0x15, SITE_CP_TE = 0x16,
-                   SITE_CP_FULL = 0x17;
+                   SITE_MMA_DRAIN = 0x13, SITE_EPI = 0x14, SITE_MMA_SF = 0x15, SITE_SF_TE = 0x16,
+                   SITE_SF_LOADED = 0x17, SITE_SF_EMPTY = 0x18;
 
 struct Params {
   const uint8_t* ascales_tiled;
@@ -110,24 +118,29 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t s_ring = smem_u32(smem);
-  auto s_a = [&](uint32_t s) { return s_ring + s * STAGE_BYTES; };
-  auto s_b = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + A_BYTES; };
-  auto s_sfa = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + A_BYTES + B_BYTES; };
-  auto s_sfb = [&](uint32_t s) {
-    return s_ring + s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES;
-  };
-  const uint32_t s_out = s_ring + RING_BYTES;
+  auto s_a = [&](uint32_t s) { return s_ring + s * AB_SLOT_BYTES; };
+  auto s_b = [&](uint32_t s) { return s_ring + s * AB_SLOT_BYTES + A_BYTES; };
+  const uint32_t s_sfring = s_ring + AB_RING_BYTES;
+  auto s_sfa = [&](uint32_t s) { return s_sfring + s * SF_SLOT_BYTES; };
+  auto s_sfb = [&](uint32_t s) { return s_sfring + s * SF_SLOT_BYTES + SFA_BYTES; };
+  const uint32_t s_out = s_sfring + SF_RING_BYTES;
   const uint32_t s_colv = s_out + OUT_BYTES;
   const uint32_t s_bar = s_colv + COLV_BYTES;
+  // barriers: operand ring full / empty, scale ring loaded / full / empty
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
-  auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
-  auto sf_full_bar = [&](uint32_t s) { return s_bar + 8u * (2 * STAGES + s); };
-  const uint32_t tmem_full_bar = s_bar + 24u * STAGES;
+  auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (AB_SLOTS + s); };
+  auto sf_loaded_bar = [&](uint32_t s) { return s_bar + 8u * (2 * AB_SLOTS + s); };
+  auto sf_full_bar = [&](uint32_t s) { return s_bar + 8u * (2 * AB_SLOTS + SF_SLOTS + s); };
+  auto sf_empty_bar = [&](uint32_t s) {
+    return s_bar + 8u * (2 * AB_SLOTS + 2 * SF_SLOTS + s);
+  };
+  const uint32_t tmem_full_bar = s_bar + 8u * (2 * AB_SLOTS + 3 * SF_SLOTS);
   const uint32_t tmem_empty_bar = tmem_full_bar + 8u;
   const uint32_t drain_bar = tmem_full_bar + 16u;
   const uint32_t final_bar = tmem_full_bar + 24u;
-  const uint32_t cp_final_bar = tmem_full_bar + 32u;
+  const uint32_t sf_final_bar = tmem_full_bar + 32u;
   const uint32_t tmem_slot = tmem_full_bar + 40u;
+  static_assert(8 * (2 * AB_SLOTS + 3 * SF_SLOTS) + 48 <= BAR_BYTES, "barriers fit");
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
 
   const int warp = threadIdx.x >> 5;
@@ -139,16 +152,20 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
     prefetch_tmap(&tm_l);
     prefetch_tmap(&tm_p);
     prefetch_tmap(&tm_y);
-    for (uint32_t s = 0; s < STAGES; ++s) {
+    for (uint32_t s = 0; s < AB_SLOTS; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
+    }
+    for (uint32_t s = 0; s < SF_SLOTS; ++s) {
+      mbar_init(sf_loaded_bar(s), 1);
       mbar_init(sf_full_bar(s), 1);
+      mbar_init(sf_empty_bar(s), 1);
     }
     mbar_init(tmem_full_bar, 1);
     mbar_init(tmem_empty_bar, NUM_EPI_WARPS);
     mbar_init(drain_bar, 1);
     mbar_init(final_bar, 1);
-    mbar_init(cp_final_bar, 1);
+    mbar_init(sf_final_bar, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -173,22 +190,16 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
         const int mb = t % p.m_tiles;
         const int nb = t / p.m_tiles;
         for (int st = 0; st < num_k + 2; ++st, ++it) {
-          const uint32_t s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
+          const uint32_t s = it % AB_SLOTS;
+          const uint32_t ph = (it / AB_SLOTS) & 1u;
           if (!svdq_wait(empty_bar(s), ph ^ 1u, SITE_PROD)) {
             ok = false;
             break;
           }
           if (st < num_k) {
-            mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES);
+            mbar_arrive_expect_tx(full_bar(s), AB_SLOT_BYTES);
             tma_load_2d(s_a(s), &tm_a, st * BK_BYTES, mb * BM, full_bar(s));
             tma_load_2d(s_b(s), &tm_b, st * BK_BYTES, nb * BN, full_bar(s));
-            bulk_load(s_sfa(s),
-                      p.ascales_tiled + (static_cast<size_t>(mb) * kblocks + 4 * st) * 512,
-                      SFA_BYTES, full_bar(s));
-            bulk_load(s_sfb(s),
-                      p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * st) * 1024,
-                      SFB_BYTES, full_bar(s));
           } else {
             const int hr = st - num_k;           // which 64-wide half of R
             mbar_arrive_expect_tx(full_bar(s), LR_A_BYTES + LR_B_BYTES);
@@ -199,10 +210,10 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
       }
       if (!ok) {
         // Let the copies already issued land before the block exits.
-        const uint32_t n = it < STAGES ? it : STAGES;
+        const uint32_t n = it < AB_SLOTS ? it : AB_SLOTS;
         for (uint32_t j = 0; j < n; ++j) {
           const uint32_t jt = it - 1 - j;
-          drain_wait(full_bar(jt % STAGES), (jt / STAGES) & 1u, 50000000ull);
+          drain_wait(full_bar(jt % AB_SLOTS), (jt / AB_SLOTS) & 1u, 50000000ull);
         }
       }
     }
@@ -211,24 +222,22 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
       // ---------------------------------------------------- MMA issuer --
       const uint32_t idesc_main = idesc_nvfp4(BM, BN);
       const uint32_t idesc_lr = idesc_bf16_f32(BM, BN, 0, 0);
-      uint32_t it = 0, tc = 0;
+      uint32_t it = 0, ik = 0, tc = 0;   // operand ring uses, K steps, tiles
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
         if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_MMA_TE)) break;
         tc_fence_after();
-        for (int st = 0; st < num_k; ++st, ++it) {
-          const uint32_t s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
-            ok = false;
-            break;
-          }
-          if (!svdq_wait(sf_full_bar(s), ph, SITE_MMA_SF)) {
+        for (int st = 0; st < num_k; ++st, ++it, ++ik) {
+          const uint32_t s = it % AB_SLOTS;
+          const uint32_t ph = (it / AB_SLOTS) & 1u;
+          const uint32_t sf = ik % SF_SLOTS;
+          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL) ||
+              !svdq_wait(sf_full_bar(sf), (ik / SF_SLOTS) & 1u, SITE_MMA_SF)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
+          const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * sf;
           const uint32_t sfb_t = sfa_t + 16;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -238,6 +247,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
                       sfa_t + 4 * j, sfb_t + 8 * j, (st | j) != 0 ? 1u : 0u);
           }
           tc_commit(empty_bar(s));
+          tc_commit(sf_empty_bar(sf));
         }
         if (!ok) break;
         // The low-rank accumulator overlaps the scale-factor columns: let
@@ -246,10 +256,9 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
         if (!svdq_wait(drain_bar, tc & 1u, SITE_MMA_DRAIN)) break;
         tc_fence_after();
         for (int hr = 0; hr < 2 && ok; ++hr, ++it) {
-          const uint32_t s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL) ||
-              !svdq_wait(sf_full_bar(s), ph, SITE_MMA_SF)) {
+          const uint32_t s = it % AB_SLOTS;
+          const uint32_t ph = (it / AB_SLOTS) & 1u;
+          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
             ok = false;
             break;
           }
@@ -269,53 +278,81 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
       tc_commit(final_bar);
       drain_wait(final_bar, 0, 100000000ull);
     }
-  } else if (warp == 2) {
+  } else if (warp == 2 || warp == 3) {
     if (lane == 0) {
-      // -------------------------------------------------- scale copier --
-      uint32_t it = 0, tc = 0;
+      // ------------------------------------------ scale-factor pipeline --
+      // K steps of this CTA, in order over its tiles: step i belongs to the
+      // tile blockIdx.x + (i / num_k) * gridDim.x, K step i % num_k.
+      const int my_tiles =
+          static_cast<int>(blockIdx.x) < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      const uint32_t total = static_cast<uint32_t>(my_tiles) * num_k;
+      uint32_t i = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
-        // The slots' scale columns overlap the low-rank accumulator: wait
-        // until the epilogue has read the previous tile.
-        if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_CP_TE)) break;
-        tc_fence_after();
-        // Every ring slot use is waited on in order, the low-rank slots
-        // included, and every use completes one phase of its slot's
-        // sf_full barrier: a parity wait is then never two phases ahead.
-        for (int st = 0; st < num_k + 2; ++st, ++it) {
-          const uint32_t s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!svdq_wait(full_bar(s), ph, SITE_CP_FULL)) {
+      if (warp == 3) {
+        // loader: slot i % SF_SLOTS is free once the MMAs of step
+        // i - SF_SLOTS (which read its TMEM columns, after the copies that
+        // read its shared memory) have completed.
+        for (; i < total; ++i) {
+          const uint32_t s = i % SF_SLOTS;
+          const uint32_t ph = (i / SF_SLOTS) & 1u;
+          if (i >= SF_SLOTS && !svdq_wait(sf_empty_bar(s), ph ^ 1u, SITE_SF_EMPTY)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          if (st < num_k) {
-            // 4 A blocks (128 rows x 64 k each), 4 x 2 halves of B blocks.
-            const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
-            const uint32_t sfb_t = sfa_t + 16;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tmem_cp_32x128b_warpx4(sfa_t + 4 * j,
-                                     smem_desc(s_sfa(s) + 512 * j, 0, 128, kLayoutSwizzleNone));
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-              for (int h = 0; h < 2; ++h)
-                tmem_cp_32x128b_warpx4(
-                    sfb_t + 8 * j + 4 * h,
-                    smem_desc(s_sfb(s) + 1024 * j + 512 * h, 0, 128, kLayoutSwizzleNone));
+          const int t = blockIdx.x + static_cast<int>(i / num_k) * gridDim.x;
+          const int st = static_cast<int>(i % num_k);
+          const int mb = t % p.m_tiles;
+          const int nb = t / p.m_tiles;
+          mbar_arrive_expect_tx(sf_loaded_bar(s), SF_SLOT_BYTES);
+          bulk_load(s_sfa(s),
+                    p.ascales_tiled + (static_cast<size_t>(mb) * kblocks + 4 * st) * 512,
+                    SFA_BYTES, sf_loaded_bar(s));
+          bulk_load(s_sfb(s),
+                    p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * st) * 1024,
+                    SFB_BYTES, sf_loaded_bar(s));
+        }
+        if (!ok) {
+          // Let the scale loads already issued land before the block exits.
+          for (uint32_t j = i > SF_SLOTS ? i - SF_SLOTS : 0; j < i; ++j)
+            drain_wait(sf_loaded_bar(j % SF_SLOTS), (j / SF_SLOTS) & 1u, 50000000ull);
+        }
+      } else {
+        // copier
+        for (; i < total; ++i) {
+          const uint32_t s = i % SF_SLOTS;
+          const uint32_t ph = (i / SF_SLOTS) & 1u;
+          if (i % num_k == 0) {
+            // The scale slots overlap the low-rank accumulator: the next
+            // tile's copies wait until the epilogue has read this tile.
+            const uint32_t tc = i / num_k;
+            if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_SF_TE)) break;
           }
+          if (!svdq_wait(sf_loaded_bar(s), ph, SITE_SF_LOADED)) break;
+          tc_fence_after();
+          // 4 A blocks (128 rows x 64 k each), 4 x 2 halves of B blocks.
+          const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
+          const uint32_t sfb_t = sfa_t + 16;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tmem_cp_32x128b_warpx4(sfa_t + 4 * j,
+                                   smem_desc(s_sfa(s) + 512 * j, 0, 128, kLayoutSwizzleNone));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tmem_cp_32x128b_warpx4(
+                  sfb_t + 8 * j + 4 * h,
+                  smem_desc(s_sfb(s) + 1024 * j + 512 * h, 0, 128, kLayoutSwizzleNone));
           tc_commit(sf_full_bar(s));
         }
+        tc_commit(sf_final_bar);
+        drain_wait(sf_final_bar, 0, 100000000ull);
       }
-      tc_commit(cp_final_bar);
-      drain_wait(cp_final_bar, 0, 100000000ull);
     }
   } else {
     // -------------------------------------------------------- epilogue --
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    const int half = (warp - EPI_WARP0) >> 2;    // which 128 of the tile's 256 columns
+    const int half = (warp - EPI_WARP0) >> 2;     // which 128 of the tile's 256 columns
     const int et = threadIdx.x - 32 * EPI_WARP0;  // 0..255
     const float alpha = __bfloat162float(p.wtscale[0]);
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
