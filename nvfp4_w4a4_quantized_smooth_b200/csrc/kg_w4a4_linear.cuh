@@ -18,17 +18,23 @@
 //               tcgen05.mma kind::mxf4nvf4 block16 (M=128, N=256, K=64) into
 //               the main accumulator, then tcgen05.mma kind::f16 (bf16,
 //               K=16) for L @ proj_up^T into a second accumulator.
-//   warps 2, 3  scale-factor pipeline: a deeper ring of SF_SLOTS slots, each
-//               one K step's A and B scale blocks (two contiguous bulk
-//               copies, 6 KB), paired with SF_SLOTS TMEM slots.  Warp 3
-//               (one thread) loads a slot as soon as the MMAs that used it
-//               have completed; warp 2 (one thread) copies each loaded slot
-//               smem -> TMEM (tcgen05.cp 32x128b.warpx4, 12 per step).  So
-//               the copies of a step are issued several steps before its
-//               MMAs and never wait on an MMA; issued from their own warp
-//               they run alongside the MMAs.
-//   warps 4..11 epilogue (two warps per TMEM lane quarter, one per half
-//               of the 256 columns): stage the tile's wcscales / bias in
+//   warp 2      scale loader (one thread): a deeper ring of SF_SLOTS slots,
+//               each one K step's A and B scale blocks (two contiguous bulk
+//               copies, 6 KB), paired with SF_SLOTS TMEM slots; a slot is
+//               reloaded as soon as the MMAs that used it have completed.
+//   warps 3..10 scale writers during the K loop, epilogue after it (two
+//               warps per TMEM lane quarter).
+//               Scale writing: the MMA reads each 512-byte scale block
+//               replicated in all four lane quarters (lane r % 32 of every
+//               quarter, column (r % 128) / 32).  Each warp reads its half
+//               of a loaded slot from shared memory (16 B per lane per
+//               block) and writes it to its quarter's lanes with
+//               tcgen05.st, several steps ahead of the MMAs.  Measured on
+//               B200, register stores from eight warps slow the
+//               concurrently running MMAs far less than tcgen05.cp copies
+//               of the same bytes.
+//               Epilogue (one warp per quarter and half of the 256
+//               columns): stage the tile's wcscales / bias in
 //               shared memory while the MMAs run, then TMEM -> registers
 //               (tcgen05.ld), fp32 acc * wtscale * wcscales + lowrank + bias,
 //               packed to bf16.  TMEM is released to the next tile right
@@ -76,7 +82,7 @@ constexpr uint32_t COLV_BYTES = 2 * 2 * BN * 4;      // wcscales, bias (fp32), 2
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BYTES =
     AB_RING_BYTES + SF_RING_BYTES + OUT_BYTES + COLV_BYTES + BAR_BYTES + 1024;
-constexpr int EPI_WARP0 = 4;
+constexpr int EPI_WARP0 = 3;
 constexpr int NUM_THREADS = 32 * EPI_WARP0 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_ACC = 0;
@@ -89,8 +95,8 @@ static_assert(AB_SLOT_BYTES % 1024 == 0 && (AB_RING_BYTES + SF_RING_BYTES) % 102
 
 // Wait-site ids recorded in the error word.
 constexpr uint32_t SITE_PROD = 0x10, SITE_MMA_TE = 0x11, SITE_MMA_FULL = 0x12,
-                   SITE_MMA_DRAIN = 0x13, SITE_EPI = 0x14, SITE_MMA_SF = 0x15, SITE_SF_TE = 0x16,
-                   SITE_SF_LOADED = 0x17, SITE_SF_EMPTY = 0x18;
+                   SITE_MMA_DRAIN = 0x13, SITE_EPI = 0x14, SITE_MMA_SF = 0x15,
+                   SITE_SF_LOADED = 0x17, SITE_SF_EMPTY = 0x18, SITE_LOAD_EMPTY = 0x19;
 
 struct Params {
   const uint8_t* ascales_tiled;
@@ -138,8 +144,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
   const uint32_t tmem_empty_bar = tmem_full_bar + 8u;
   const uint32_t drain_bar = tmem_full_bar + 16u;
   const uint32_t final_bar = tmem_full_bar + 24u;
-  const uint32_t sf_final_bar = tmem_full_bar + 32u;
-  const uint32_t tmem_slot = tmem_full_bar + 40u;
+  const uint32_t tmem_slot = tmem_full_bar + 32u;
   static_assert(8 * (2 * AB_SLOTS + 3 * SF_SLOTS) + 48 <= BAR_BYTES, "barriers fit");
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
 
@@ -158,14 +163,13 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
     }
     for (uint32_t s = 0; s < SF_SLOTS; ++s) {
       mbar_init(sf_loaded_bar(s), 1);
-      mbar_init(sf_full_bar(s), 1);
+      mbar_init(sf_full_bar(s), NUM_EPI_WARPS);
       mbar_init(sf_empty_bar(s), 1);
     }
     mbar_init(tmem_full_bar, 1);
     mbar_init(tmem_empty_bar, NUM_EPI_WARPS);
     mbar_init(drain_bar, 1);
     mbar_init(final_bar, 1);
-    mbar_init(sf_final_bar, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -278,75 +282,40 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
       tc_commit(final_bar);
       drain_wait(final_bar, 0, 100000000ull);
     }
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp == 2) {
     if (lane == 0) {
-      // ------------------------------------------ scale-factor pipeline --
+      // -------------------------------------------------- scale loader --
       // K steps of this CTA, in order over its tiles: step i belongs to the
       // tile blockIdx.x + (i / num_k) * gridDim.x, K step i % num_k.
+      // Slot i % SF_SLOTS is free once the MMAs of step i - SF_SLOTS (which
+      // read its TMEM columns, written from its shared memory) completed.
       const int my_tiles =
           static_cast<int>(blockIdx.x) < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
       const uint32_t total = static_cast<uint32_t>(my_tiles) * num_k;
       uint32_t i = 0;
       bool ok = true;
-      if (warp == 3) {
-        // loader: slot i % SF_SLOTS is free once the MMAs of step
-        // i - SF_SLOTS (which read its TMEM columns, after the copies that
-        // read its shared memory) have completed.
-        for (; i < total; ++i) {
-          const uint32_t s = i % SF_SLOTS;
-          const uint32_t ph = (i / SF_SLOTS) & 1u;
-          if (i >= SF_SLOTS && !svdq_wait(sf_empty_bar(s), ph ^ 1u, SITE_SF_EMPTY)) {
-            ok = false;
-            break;
-          }
-          const int t = blockIdx.x + static_cast<int>(i / num_k) * gridDim.x;
-          const int st = static_cast<int>(i % num_k);
-          const int mb = t % p.m_tiles;
-          const int nb = t / p.m_tiles;
-          mbar_arrive_expect_tx(sf_loaded_bar(s), SF_SLOT_BYTES);
-          bulk_load(s_sfa(s),
-                    p.ascales_tiled + (static_cast<size_t>(mb) * kblocks + 4 * st) * 512,
-                    SFA_BYTES, sf_loaded_bar(s));
-          bulk_load(s_sfb(s),
-                    p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * st) * 1024,
-                    SFB_BYTES, sf_loaded_bar(s));
+      for (; i < total; ++i) {
+        const uint32_t s = i % SF_SLOTS;
+        const uint32_t ph = (i / SF_SLOTS) & 1u;
+        if (i >= SF_SLOTS && !svdq_wait(sf_empty_bar(s), ph ^ 1u, SITE_LOAD_EMPTY)) {
+          ok = false;
+          break;
         }
-        if (!ok) {
-          // Let the scale loads already issued land before the block exits.
-          for (uint32_t j = i > SF_SLOTS ? i - SF_SLOTS : 0; j < i; ++j)
-            drain_wait(sf_loaded_bar(j % SF_SLOTS), (j / SF_SLOTS) & 1u, 50000000ull);
-        }
-      } else {
-        // copier
-        for (; i < total; ++i) {
-          const uint32_t s = i % SF_SLOTS;
-          const uint32_t ph = (i / SF_SLOTS) & 1u;
-          if (i % num_k == 0) {
-            // The scale slots overlap the low-rank accumulator: the next
-            // tile's copies wait until the epilogue has read this tile.
-            const uint32_t tc = i / num_k;
-            if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_SF_TE)) break;
-          }
-          if (!svdq_wait(sf_loaded_bar(s), ph, SITE_SF_LOADED)) break;
-          tc_fence_after();
-          // 4 A blocks (128 rows x 64 k each), 4 x 2 halves of B blocks.
-          const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
-          const uint32_t sfb_t = sfa_t + 16;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tmem_cp_32x128b_warpx4(sfa_t + 4 * j,
-                                   smem_desc(s_sfa(s) + 512 * j, 0, 128, kLayoutSwizzleNone));
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tmem_cp_32x128b_warpx4(
-                  sfb_t + 8 * j + 4 * h,
-                  smem_desc(s_sfb(s) + 1024 * j + 512 * h, 0, 128, kLayoutSwizzleNone));
-          tc_commit(sf_full_bar(s));
-        }
-        tc_commit(sf_final_bar);
-        drain_wait(sf_final_bar, 0, 100000000ull);
+        const int t = blockIdx.x + static_cast<int>(i / num_k) * gridDim.x;
+        const int st = static_cast<int>(i % num_k);
+        const int mb = t % p.m_tiles;
+        const int nb = t / p.m_tiles;
+        mbar_arrive_expect_tx(sf_loaded_bar(s), SF_SLOT_BYTES);
+        bulk_load(s_sfa(s), p.ascales_tiled + (static_cast<size_t>(mb) * kblocks + 4 * st) * 512,
+                  SFA_BYTES, sf_loaded_bar(s));
+        bulk_load(s_sfb(s),
+                  p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * st) * 1024,
+                  SFB_BYTES, sf_loaded_bar(s));
+      }
+      if (!ok) {
+        // Let the scale loads already issued land before the block exits.
+        for (uint32_t j = i > SF_SLOTS ? i - SF_SLOTS : 0; j < i; ++j)
+          drain_wait(sf_loaded_bar(j % SF_SLOTS), (j / SF_SLOTS) & 1u, 50000000ull);
       }
     }
   } else {
@@ -358,11 +327,40 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t s_obuf = s_out + static_cast<uint32_t>(warp - EPI_WARP0) * OUT_WARP_BYTES;
     float* colv = reinterpret_cast<float*>(smem + (s_colv - s_ring));
-    uint32_t tc = 0;
+    uint32_t tc = 0, i = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
       const int mb = t % p.m_tiles;
       const int nb = t / p.m_tiles;
+      // Scale factors of this tile's K steps -> TMEM, up to SF_SLOTS steps
+      // ahead of the MMAs.  This warp writes blocks 6 * half .. 6 * half + 5
+      // of each slot (TMEM columns 4 b .. 4 b + 3 for block b) in its lane
+      // quarter.  The previous tile's epilogue, above in program order, has
+      // already read the low-rank accumulator these columns overlap.
+      for (int st = 0; st < num_k; ++st, ++i) {
+        const uint32_t s = i % SF_SLOTS;
+        const uint32_t ph = (i / SF_SLOTS) & 1u;
+        if (ok)
+          ok = __all_sync(0xFFFFFFFFu,
+                          svdq_wait(sf_loaded_bar(s), ph, SITE_SF_LOADED) &&
+                              (i < SF_SLOTS || svdq_wait(sf_empty_bar(s), ph ^ 1u, SITE_SF_EMPTY)));
+        if (!ok) continue;
+        tc_fence_after();
+        const uint32_t src = s_sfa(s) + 16 * lane;
+        const uint32_t dst = lane_base + TM_SF + TM_SF_SLOT * s;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const int b0 = 6 * half + 2 * k;
+          uint32_t v[8];
+          ld_shared_v4(src + 512 * b0, v[0], v[1], v[2], v[3]);
+          ld_shared_v4(src + 512 * (b0 + 1), v[4], v[5], v[6], v[7]);
+          tmem_st_32x32b_x8(dst + 4 * b0, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_full_bar(s));
+      }
       // Per-column factors of this tile -> shared memory (double buffered by
       // tile parity), loaded while the tile's MMAs are still running.
       float* wc_s = colv + (tc & 1u) * (2 * BN);
@@ -434,6 +432,9 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
   }
 
   // ----------------------------------------------------------- teardown --
+  // Role loops run in one lane of some warps: reconverge every warp first,
+  // so that the block barrier waits for all of its threads.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -469,6 +469,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   }
 
   // ----------------------------------------------------------- teardown --
+  // Role loops run in one lane of some warps: reconverge every warp first,
+  // so that the block barrier waits for all of its threads.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
