@@ -96,7 +96,8 @@ static_assert(AB_SLOT_BYTES % 1024 == 0 && (AB_RING_BYTES + SF_RING_BYTES) % 102
 // Wait-site ids recorded in the error word.
 constexpr uint32_t SITE_PROD = 0x10, SITE_MMA_TE = 0x11, SITE_MMA_FULL = 0x12,
                    SITE_MMA_DRAIN = 0x13, SITE_EPI = 0x14, SITE_MMA_SF = 0x15,
-                   SITE_SF_LOADED = 0x17, SITE_SF_EMPTY = 0x18, SITE_LOAD_EMPTY = 0x19;
+                   SITE_SF_LOADED = 0x17, SITE_SF_EMPTY = 0x18, SITE_LOAD_EMPTY = 0x19,
+                   SITE_EPI_TE = 0x1A;
 
 struct Params {
   const uint8_t* ascales_tiled;
@@ -329,15 +330,14 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
     float* colv = reinterpret_cast<float*>(smem + (s_colv - s_ring));
     uint32_t tc = 0, i = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
-      const int mb = t % p.m_tiles;
-      const int nb = t / p.m_tiles;
-      // Scale factors of this tile's K steps -> TMEM, up to SF_SLOTS steps
-      // ahead of the MMAs.  This warp writes blocks 6 * half .. 6 * half + 5
-      // of each slot (TMEM columns 4 b .. 4 b + 3 for block b) in its lane
-      // quarter.  The previous tile's epilogue, above in program order, has
-      // already read the low-rank accumulator these columns overlap.
-      for (int st = 0; st < num_k; ++st, ++i) {
+    // Scale factors of the next n K steps -> TMEM, up to SF_SLOTS steps
+    // ahead of the MMAs.  This warp writes blocks 6 * half .. 6 * half + 5
+    // of each slot (TMEM columns 4 b .. 4 b + 3 for block b) in its lane
+    // quarter.  A tile's steps are written only after every epilogue warp
+    // has read the previous tile's low-rank accumulator, which these
+    // columns overlap.
+    auto write_scales = [&](uint32_t n) {
+      for (uint32_t e = i + n; i < e; ++i) {
         const uint32_t s = i % SF_SLOTS;
         const uint32_t ph = (i / SF_SLOTS) & 1u;
         if (ok)
@@ -361,6 +361,20 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
         __syncwarp();
         if (lane == 0) mbar_arrive(sf_full_bar(s));
       }
+    };
+    // A tile's first SF_SLOTS steps are written right after the previous
+    // tile's TMEM reads, before its output stores, and MID more between the
+    // two output pieces, so the MMAs restart soon and do not wait for the
+    // stores.
+    constexpr uint32_t MID = 2;
+    const uint32_t head = num_k < SF_SLOTS ? static_cast<uint32_t>(num_k) : SF_SLOTS;
+    const uint32_t mid = num_k - head < MID ? num_k - head : MID;
+    if (static_cast<int>(blockIdx.x) < tiles) write_scales(head + mid);
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
+      const int mb = t % p.m_tiles;
+      const int nb = t / p.m_tiles;
+      const bool has_next = t + static_cast<int>(gridDim.x) < tiles;
+      write_scales(num_k - head - mid);
       // Per-column factors of this tile -> shared memory (double buffered by
       // tile parity), loaded while the tile's MMAs are still running.
       float* wc_s = colv + (tc & 1u) * (2 * BN);
@@ -404,6 +418,12 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tmem_empty_bar);
+      if (has_next) {
+        // The other warp of this lane quarter may still be reading low-rank
+        // columns that the next scale slots overlap: wait for all readers.
+        ok = __all_sync(0xFFFFFFFFu, svdq_wait(tmem_empty_bar, tc & 1u, SITE_EPI_TE));
+        write_scales(head);
+      }
       // Rows -> swizzled buffer (row = lane, 128 B per row; 16-byte chunk
       // j of row r at chunk j ^ (r % 8), the TMA 128-byte swizzle) -> TMA
       // store of 32 rows x 64 columns, twice per tile.
@@ -426,6 +446,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
           tma_store_2d(&tm_y, s_obuf, x0, row0);
           bulk_commit_group();
         }
+        if (pc == 0 && has_next) write_scales(mid);
       }
     }
     if (lane == 0) bulk_wait_group0();
