@@ -12,35 +12,43 @@
 //   q = E2M1(v / s)                 quotient, then the hardware RNE /
 //                                   satfinite conversion
 // Each quotient a / b is formed as r = 1/b (reciprocal), q0 = a r, then one
-// residual step e = a - q0 b (exact by FMA), q = q0 + e r (Markstein, IBM J.
-// Res. Dev. 34(1), 1990).  Rounding that q equals rounding the exact
-// quotient: a bf16 x bf16 product has at most 16 significant bits, and
-// every e4m3 midpoint x 6 and every E2M1 midpoint x s at most 7, so a
-// quotient that is not exactly a midpoint lies at least 2^-16 (relative)
-// from it, far more than q's error (a few ulps of fp32); a quotient that is
-// exactly a midpoint is representable and the residual step returns it
-// exactly (|1 - b r| <= 2^-22 makes the step's error far below half an
-// ulp), so the conversion sees the tie.  A scale that rounds to zero gives
-// r = 0 and therefore signed zero codes.
+// residual step (Markstein, IBM J. Res. Dev. 34(1), 1990) with the residual
+// exact by FMA.  Rounding that q equals rounding the exact quotient: a
+// bf16 x bf16 product has at most 16 significant bits, and every e4m3
+// midpoint x 6 and every E2M1 midpoint x s at most 7, so a quotient that is
+// not exactly a midpoint lies at least 2^-16 (relative) from it, far more
+// than q's error (a few ulps of fp32); a quotient that is exactly a
+// midpoint is representable and the residual step returns it exactly
+// (|1 - b r| <= 2^-22 makes the step's error far below half an ulp), so the
+// conversion sees the tie.
+// The element quotients are computed on nv = x * (-smooth) = -v with the
+// negated reciprocal: q0 = nv (-r) = v r, e = q0 s + nv = q0 s - v,
+// q = q0 + e (-r).  These are the same roundings as q0 = v r,
+// e = v - q0 s, q = q0 + e r, and they also keep the sign of a zero v
+// (v = -0 gives q0 = -0, e = +0, q = -0; v = +0 gives +0), which the E2M1
+// code must carry.  A scale that rounds to zero gives -r = -0 and therefore
+// signed zero codes.
 //
-// CTA layout: a tile of BM rows (32..256) over a K range, 18 warps.
-//   warp 0      TMA producer: per stage of 64 or 128 k, the x tile as
-//               [BM rows x 64 k] bf16 boxes (128-byte swizzle), proj_down
-//               rows [64 k x 128 r] per box pair (64 x 64 boxes) and the
-//               smooth values, into a ring of stages.
+// CTA work item: a tile of BM = 128 rows and one of `split` ranges of K.
+// 18 warps:
+//   warp 0      TMA producer: per stage of 128 k, the x tile (one 3-D box:
+//               2 chunks x [128 rows x 64 k] bf16, 128-byte swizzle), the
+//               proj_down rows (one 3-D box: 2 halves of 64 r x [128 k x
+//               128 B]) and 256 B of smooth, into a ring of 3 stages.
 //   warp 1      TMEM owner, MMA issuer.  The low-rank product is computed
-//               transposed, L^T[128 x BM] += proj_down_chunk^T x_tile^T:
-//               tcgen05.mma kind::f16, M = 128 (= R), N = BM, K = 16;
-//               A (proj_down) MN-major, B (x tile) K-major, fp32 in BM
-//               TMEM columns.  So BM is free (multiple of 32) while the
-//               accumulator keeps the full 128-lane layout.
-//   warps 2..17 quantize the same shared-memory x tile (four warps per
-//               scheduler, one 16-element group per thread per stage for
-//               BM = 64), write packed codes and tiled scales; afterwards
-//               read L^T out of TMEM.
-// The K range is split over a thread-block cluster of `split` CTAs; the
-// partial L tiles are summed through distributed shared memory in rank
-// order (deterministic) and written once as bf16.
+//               transposed, L^T[128 x 128] += proj_down_stage^T x_tile^T:
+//               tcgen05.mma kind::f16, M = 128 (= R), N = 128 (rows),
+//               K = 16; A (proj_down) MN-major, B (x tile) K-major, fp32
+//               accumulator in 128 TMEM columns.
+//   warps 2..17 quantizers: thread t owns 16-element group (t % 8) of the
+//               stage's 128 k and rows t / 8 and t / 8 + 64, so it converts
+//               its 16 smooth values once per stage and runs two
+//               independent groups side by side; writes packed codes and
+//               tiled scales; afterwards reads L^T out of TMEM.
+// With split == 1 the tile's L is rounded to bf16 and written directly.
+// Otherwise each CTA writes its fp32 partial to the workspace and counts
+// itself in; the last CTA of a row tile sums the split partials in K order
+// (deterministic), writes bf16 L and resets the tile's counter to zero.
 #pragma once
 
 #include <cuda.h>
@@ -53,72 +61,47 @@ namespace svdq {
 namespace kq {
 
 constexpr int R = 128;                 // rank (MMA M)
+constexpr int BM = 128;                // rows per tile (MMA N)
 constexpr int BKE = 64;                // k per chunk (one 128-byte swizzled box row)
-constexpr int MAX_BM = 256;
-constexpr int MAX_STAGES = 6;
-constexpr uint32_t PD_BOX = 64 * 64 * 2;          // [64 k x 64 r] bf16 box, 8 KB
-constexpr uint32_t PD_CHUNK = 2 * PD_BOX;         // one chunk of proj_down, 16 KB
-constexpr uint32_t SMOOTH_CHUNK = BKE * 2;        // 128 B
+constexpr int STAGE_K = 128;           // k per stage (2 chunks)
+constexpr int STAGES = 3;
+constexpr uint32_t X_CHUNK = BM * 128;             // [128 rows x 64 k] bf16, 16 KB
+constexpr uint32_t X_BYTES = 2 * X_CHUNK;          // 32 KB
+constexpr uint32_t PD_HALF = STAGE_K * 128;        // [128 k x 64 r] bf16, 16 KB
+constexpr uint32_t PD_BYTES = 2 * PD_HALF;         // 32 KB
+constexpr uint32_t SM_BYTES = STAGE_K * 2;         // 256 B
+constexpr uint32_t STAGE_BYTES = (X_BYTES + PD_BYTES + SM_BYTES + 1023u) & ~1023u;
 constexpr int NUM_QWARPS = 16;
 constexpr int NUM_QTHREADS = NUM_QWARPS * 32;
 constexpr int NUM_THREADS = 64 + NUM_QTHREADS;
-constexpr uint32_t BAR_BYTES = 256;
-constexpr uint32_t SMEM_BUDGET = 227 * 1024;
-constexpr int PART_STRIDE = R + 4;  // floats per row m of the partial-L buffer
+constexpr uint32_t BAR_BYTES = 128;
+constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr uint32_t TMEM_COLS = 128;
+constexpr uint32_t PART_BYTES = BM * R * 4;        // one fp32 partial tile, 64 KB
+constexpr int MAX_SPLIT_TILES = 1024;              // row tiles that may split K
+constexpr uint32_t COUNTER_BYTES = MAX_SPLIT_TILES * 4;   // workspace counter area
 
 constexpr uint32_t SITE_PROD = 0x20, SITE_MMA = 0x21, SITE_QUANT = 0x22, SITE_LFULL = 0x23;
-
-// A stage holds `cps` chunks of 64 k (1 or 2): x [bm rows x 128 B] per
-// chunk, proj_down [64 k x 128 r] per chunk, 128 B of smooth per chunk.
-__host__ __device__ constexpr uint32_t x_chunk(int bm) { return static_cast<uint32_t>(bm) * 128u; }
-__host__ __device__ constexpr uint32_t x_bytes(int bm, int cps) { return cps * x_chunk(bm); }
-__host__ __device__ constexpr uint32_t stage_bytes(int bm, int cps) {
-  return (cps * (x_chunk(bm) + PD_CHUNK + SMOOTH_CHUNK) + 1023u) & ~1023u;
-}
-__host__ __device__ constexpr int num_stages(int bm, int cps) {
-  return (SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm, cps) < MAX_STAGES
-             ? static_cast<int>((SMEM_BUDGET - 1024 - BAR_BYTES) / stage_bytes(bm, cps))
-             : MAX_STAGES;
-}
-__host__ __device__ constexpr uint32_t smem_bytes(int bm, int cps) {
-  return num_stages(bm, cps) * stage_bytes(bm, cps) + BAR_BYTES + 1024;
-}
-// Two chunks per stage when that still leaves three stages in flight.
-__host__ __device__ constexpr int chunks_per_stage(int bm) {
-  return num_stages(bm, 2) >= 3 ? 2 : 1;
-}
-__host__ __device__ constexpr uint32_t tmem_cols(int bm) {
-  return bm <= 32 ? 32u : bm <= 64 ? 64u : bm <= 128 ? 128u : 256u;
-}
-static_assert(MAX_BM * PART_STRIDE * 4 <=
-                  num_stages(MAX_BM, chunks_per_stage(MAX_BM)) *
-                      stage_bytes(MAX_BM, chunks_per_stage(MAX_BM)),
-              "partial buffer fits the ring");
-static_assert(num_stages(32, chunks_per_stage(32)) >= 3 &&
-                  num_stages(MAX_BM, chunks_per_stage(MAX_BM)) >= 3,
-              "at least three stages");
 
 struct Params {
   const __nv_bfloat16* smooth;
   uint8_t* qact;
   uint8_t* ascales_tiled;
   __nv_bfloat16* lowrank;
+  float* partials;        // [split][m_tiles][BM][R] fp32 (split > 1)
+  uint32_t* counters;     // [m_tiles], zero between launches (split > 1)
   int M, K;
-  int chunks;  // K / 64
-  int split;   // CTAs per cluster along K
-  int bm;      // rows per CTA (multiple of 32, <= 256)
+  int chunks;   // K / 64
+  int split;    // K ranges per row tile
+  int m_tiles;
 };
 
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr));
   return v;
-}
-
-__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
-  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 // Packed pairs of fp32 (lo in the low word) and their arithmetic.
@@ -151,17 +134,19 @@ __device__ __forceinline__ uint64_t bf16x2_to_pk(uint32_t w) {
   return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-// One 16-element group: x (8 bf16x2 words), smooth (8 bf16x2 words) ->
-// 16 E2M1 codes (element 0 in the lowest nibble) and the e4m3 scale byte.
-__device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8], const uint32_t (&sw)[8],
+// One 16-element group: x (8 bf16x2 words) and the negated smooth values
+// as packed fp32 pairs -> 16 E2M1 codes (element 0 in the lowest nibble)
+// and the e4m3 scale byte.
+__device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
+                                                   const uint64_t (&nsm)[8],
                                                    uint32_t& scale_byte) {
-  uint64_t v[8];
+  uint64_t nv[8];
   float m8[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    v[i] = mul2(bf16x2_to_pk(xw[i]), bf16x2_to_pk(sw[i]));
+    nv[i] = mul2(bf16x2_to_pk(xw[i]), nsm[i]);
     float lo, hi;
-    upk(v[i], lo, hi);
+    upk(nv[i], lo, hi);
     m8[i] = fmaxf(fabsf(lo), fabsf(hi));
   }
   // max is exact, so a tree gives the same amax with a short dependency chain
@@ -174,23 +159,16 @@ __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8], cons
   const uint32_t sc = cvt_e4m3x2(a6, 0.0f) & 0xFFu;
   scale_byte = sc;
   const float d = e4m3_to_f32(sc);
-  const float r = d > 0.0f ? rcp_approx(d) : 0.0f;
-  const uint64_t r2 = pk(r, r);
-  const uint64_t nd2 = pk(-d, -d);
+  const float nr = d > 0.0f ? -rcp_approx(d) : -0.0f;
+  const uint64_t nr2 = pk(nr, nr);
+  const uint64_t d2 = pk(d, d);
   float q[16];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint64_t q0 = mul2(v[i], r2);
-    const uint64_t e = fma2(q0, nd2, v[i]);
-    const uint64_t q1 = fma2(e, r2, q0);
-    float lo, hi, vlo, vhi;
-    upk(q1, lo, hi);
-    upk(v[i], vlo, vhi);
-    // The residual step turns a quotient of -0 into +0: restore v's sign.
-    q[2 * i] = __uint_as_float((__float_as_uint(lo) & 0x7FFFFFFFu) |
-                               (__float_as_uint(vlo) & 0x80000000u));
-    q[2 * i + 1] = __uint_as_float((__float_as_uint(hi) & 0x7FFFFFFFu) |
-                                   (__float_as_uint(vhi) & 0x80000000u));
+    const uint64_t q0 = mul2(nv[i], nr2);       // v r
+    const uint64_t e = fma2(q0, d2, nv[i]);     // q0 s - v, exact
+    const uint64_t q1 = fma2(e, nr2, q0);       // q0 + (v - q0 s) r
+    upk(q1, q[2 * i], q[2 * i + 1]);
   }
   const float(&qlo)[8] = *reinterpret_cast<const float(*)[8]>(q);
   const float(&qhi)[8] = *reinterpret_cast<const float(*)[8]>(q + 8);
@@ -198,49 +176,42 @@ __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8], cons
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] bf16, box {64, bm}
-                    const __grid_constant__ CUtensorMap tm_pd,   // proj_down [K, 128], box {64, 64}
+quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/64}, box {64, 128, 2}
+                    const __grid_constant__ CUtensorMap tm_pd,   // proj_down {64, K, 2}, box {64, 128, 2}
                     const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int bm = p.bm;
-  const int cps = chunks_per_stage(bm);
-  const uint32_t sbytes = stage_bytes(bm, cps);
-  const uint32_t nst = static_cast<uint32_t>(num_stages(bm, cps));
   const uint32_t s_ring = smem_u32(smem);
-  const uint32_t s_bar = s_ring + nst * sbytes;
-  // Stage layout: x chunks [cps][bm rows x 128 B], proj_down chunks
-  // [cps][r half][64 k x 128 B], smooth chunks [cps][128 B].
-  auto s_x = [&](uint32_t s, int c) { return s_ring + s * sbytes + c * x_chunk(bm); };
-  auto s_pd = [&](uint32_t s, int c) {
-    return s_ring + s * sbytes + x_bytes(bm, cps) + c * PD_CHUNK;
-  };
-  auto s_sm = [&](uint32_t s, int c) {
-    return s_ring + s * sbytes + x_bytes(bm, cps) + cps * PD_CHUNK + c * SMOOTH_CHUNK;
-  };
+  const uint32_t s_bar = s_ring + STAGES * STAGE_BYTES;
+  // Stage layout: x [chunk][128 rows x 128 B], proj_down [r half][128 k x
+  // 128 B], smooth [128 k] bf16.
+  auto s_x = [&](uint32_t s) { return s_ring + s * STAGE_BYTES; };
+  auto s_pd = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + X_BYTES; };
+  auto s_sm = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + X_BYTES + PD_BYTES; };
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
-  auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (MAX_STAGES + s); };
-  const uint32_t lfull_bar = s_bar + 16u * MAX_STAGES;
+  auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
+  const uint32_t lfull_bar = s_bar + 16u * STAGES;
   const uint32_t final_bar = lfull_bar + 8u;
-  const uint32_t tmem_slot = lfull_bar + 16u;
+  const uint32_t flag_slot = lfull_bar + 16u;
+  const uint32_t tmem_slot = lfull_bar + 20u;
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
-  const uint32_t ncols = tmem_cols(bm);
+  volatile uint32_t* flag_ptr = reinterpret_cast<volatile uint32_t*>(smem + (flag_slot - s_ring));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mb = blockIdx.y;
-  const int rank = blockIdx.x;  // == rank in the cluster (cluster dims = (split, 1, 1))
-  const int c_begin = rank * p.chunks / p.split;
-  const int c_end = (rank + 1) * p.chunks / p.split;
-  // >= 1 chunk per CTA (host guarantees split <= chunks); stages of cps
-  // chunks, the last one possibly partial.
-  const int nstages = (c_end - c_begin + cps - 1) / cps;
+  const int mb = blockIdx.x % p.m_tiles;
+  const int ks = blockIdx.x / p.m_tiles;
+  const int c_begin = ks * p.chunks / p.split;      // in chunks of 64 k
+  const int c_end = (ks + 1) * p.chunks / p.split;
+  // >= 1 chunk per CTA (host guarantees split <= chunks); the last stage of
+  // a range may hold one chunk.
+  const int nstages = (c_end - c_begin + 1) / 2;
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_pd);
-    for (uint32_t s = 0; s < nst; ++s) {
+    for (uint32_t s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1 + NUM_QWARPS);
     }
@@ -249,7 +220,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, ncols);
+    tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -257,64 +228,59 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
 
-  bool l_ready = false;  // quantizer threads: L accumulator readable
-
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ producer --
       int i = 0;
       bool ok = true;
       for (; i < nstages; ++i) {
-        const uint32_t s = static_cast<uint32_t>(i) % nst;
-        const uint32_t ph = (static_cast<uint32_t>(i) / nst) & 1u;
+        const uint32_t s = static_cast<uint32_t>(i) % STAGES;
+        const uint32_t ph = (static_cast<uint32_t>(i) / STAGES) & 1u;
         if (!svdq_wait(empty_bar(s), ph ^ 1u, SITE_PROD)) {
           ok = false;
           break;
         }
-        const int kc0 = c_begin + cps * i;
-        const int nc = c_end - kc0 < cps ? c_end - kc0 : cps;
-        mbar_arrive_expect_tx(full_bar(s), nc * (x_chunk(bm) + PD_CHUNK + SMOOTH_CHUNK));
-        for (int c = 0; c < nc; ++c) {
-          const int kc = kc0 + c;
-          tma_load_2d(s_x(s, c), &tm_x, kc * BKE, mb * bm, full_bar(s));
-          tma_load_2d(s_pd(s, c), &tm_pd, 0, kc * BKE, full_bar(s));
-          tma_load_2d(s_pd(s, c) + PD_BOX, &tm_pd, 64, kc * BKE, full_bar(s));
-          bulk_load(s_sm(s, c), p.smooth + kc * BKE, SMOOTH_CHUNK, full_bar(s));
-        }
+        const int kc0 = c_begin + 2 * i;
+        const int nc = c_end - kc0 < 2 ? 1 : 2;
+        // Boxes are always delivered whole (zero fill past M and K); only
+        // the smooth copy is cut to the chunks that exist.
+        mbar_arrive_expect_tx(full_bar(s), X_BYTES + PD_BYTES + nc * 128u);
+        tma_load_3d(s_x(s), &tm_x, 0, mb * BM, kc0, full_bar(s));
+        tma_load_3d(s_pd(s), &tm_pd, 0, kc0 * BKE, 0, full_bar(s));
+        bulk_load(s_sm(s), p.smooth + kc0 * BKE, nc * 128u, full_bar(s));
       }
       if (!ok) {
-        const int n = i < static_cast<int>(nst) ? i : static_cast<int>(nst);
+        const int n = i < STAGES ? i : STAGES;
         for (int j = 0; j < n; ++j) {
           const uint32_t jt = static_cast<uint32_t>(i - 1 - j);
-          drain_wait(full_bar(jt % nst), (jt / nst) & 1u, 50000000ull);
+          drain_wait(full_bar(jt % STAGES), (jt / STAGES) & 1u, 50000000ull);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------- MMA issuer --
-      // L^T[r, m] += sum_k proj_down[k, r] x[m, k]: A = proj_down chunk
-      // (MN-major: r contiguous; the two 64-r halves are 8 KB apart, 8-row
-      // k groups 1 KB apart), B = x chunk (K-major, 128-byte rows).
-      const uint32_t idesc = idesc_bf16_f32(R, static_cast<uint32_t>(bm), 1, 0);
+      // L^T[r, m] += sum_k proj_down[k, r] x[m, k]: A = proj_down stage
+      // (MN-major: r contiguous; the two 64-r halves 16 KB apart, 8-row k
+      // groups 1 KB apart), B = x chunk (K-major, 128-byte rows).
+      const uint32_t idesc = idesc_bf16_f32(R, BM, 1, 0);
       bool ok = true;
       for (int i = 0; i < nstages; ++i) {
-        const uint32_t s = static_cast<uint32_t>(i) % nst;
-        const uint32_t ph = (static_cast<uint32_t>(i) / nst) & 1u;
+        const uint32_t s = static_cast<uint32_t>(i) % STAGES;
+        const uint32_t ph = (static_cast<uint32_t>(i) / STAGES) & 1u;
         if (!svdq_wait(full_bar(s), ph, SITE_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int kc0 = c_begin + cps * i;
-        const int nc = c_end - kc0 < cps ? c_end - kc0 : cps;
-        for (int c = 0; c < nc; ++c) {
-#pragma unroll
-          for (int kk = 0; kk < BKE / 16; ++kk) {
-            mma_f16(tmem_base, smem_desc(s_pd(s, c) + 2048 * kk, PD_BOX, 1024, kLayoutSwizzle128B),
-                    smem_desc(s_x(s, c) + 32 * kk, 16, 1024, kLayoutSwizzle128B), idesc,
-                    (i | c | kk) != 0 ? 1u : 0u);
-          }
+        const int kc0 = c_begin + 2 * i;
+        const int nk = c_end - kc0 < 2 ? 4 : 8;   // K = 16 steps in the stage
+        for (int kk = 0; kk < nk; ++kk) {
+          mma_f16(tmem_base,
+                  smem_desc(s_pd(s) + 2048 * kk, PD_HALF, 1024, kLayoutSwizzle128B),
+                  smem_desc(s_x(s) + (kk >> 2) * X_CHUNK + 32 * (kk & 3), 16, 1024,
+                            kLayoutSwizzle128B),
+                  idesc, (i | kk) != 0 ? 1u : 0u);
         }
         tc_commit(empty_bar(s));
       }
@@ -325,147 +291,135 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   } else {
     // -------------------------------------------------------- quantizers --
     const int qt = threadIdx.x - 64;
+    const int cg = qt & 7;          // group of 16 within the stage's 128 k
+    const int c = cg >> 2;          // chunk
+    const int g = cg & 3;           // group within the chunk
+    const int r0 = qt >> 3;         // rows r0 and r0 + 64 of the tile
     const int half_k = p.K / 2;
-    const int rows_pad = (p.M + 127) & ~127;   // rows the tiled scale buffer holds
+    // swizzled 16-byte x chunk positions of this group (same for both rows)
+    const uint32_t xo0 =
+        static_cast<uint32_t>(c) * X_CHUNK + r0 * 128 + ((((2 * g) ^ r0) & 7) << 4);
+    const uint32_t xo1 =
+        static_cast<uint32_t>(c) * X_CHUNK + r0 * 128 + ((((2 * g + 1) ^ r0) & 7) << 4);
+    const int m0 = mb * BM + r0;
+    const int m1 = m0 + 64;
+    uint8_t* q0_row = p.qact + static_cast<size_t>(m0) * half_k + g * 8;
+    uint8_t* q1_row = p.qact + static_cast<size_t>(m1) * half_k + g * 8;
+    // tiled scales: 512-byte block per (128 rows, 64 k); byte
+    // (row % 32) * 16 + ((row % 128) / 32) * 4 + group
+    uint8_t* sc_base = p.ascales_tiled + static_cast<size_t>(mb) * p.chunks * 512;
+    const uint32_t sc_off0 = (r0 & 31) * 16 + (r0 >> 5) * 4;
+    const uint32_t sc_off1 = (r0 & 31) * 16 + ((r0 + 64) >> 5) * 4;
     bool ok = true;
     for (int i = 0; i < nstages; ++i) {
-      const uint32_t s = static_cast<uint32_t>(i) % nst;
-      const uint32_t ph = (static_cast<uint32_t>(i) / nst) & 1u;
+      const uint32_t s = static_cast<uint32_t>(i) % STAGES;
+      const uint32_t ph = (static_cast<uint32_t>(i) / STAGES) & 1u;
       if (!__all_sync(0xFFFFFFFFu, svdq_wait(full_bar(s), ph, SITE_QUANT))) {
         ok = false;
         break;
       }
-      const int kc0 = c_begin + cps * i;
-      const int nc = c_end - kc0 < cps ? c_end - kc0 : cps;
-      // bm rows x (4 cps) groups; consecutive lanes take one row's groups
-      // (chunk c, then group g of 16 within it), whole warps together.
-      const int gshift = cps == 2 ? 3 : 2;   // log2(groups per row per stage)
-      for (int gi = qt; gi < (bm << gshift); gi += NUM_QTHREADS) {
-        const int r = gi >> gshift;               // row in the tile
-        const int c = (gi >> 2) & (cps - 1);      // chunk within the stage
-        const int g = gi & 3;                     // group of 16 within the chunk
-        const bool active = c < nc;     // the stage's second chunk may be absent
-        const int row = mb * bm + r;
-        const int kc = kc0 + c;
-        uint32_t scale = 0;
-        if (active) {
-          const uint32_t row_addr = s_x(s, c) + r * 128;
-          const uint4 xa = ld_shared_v4(row_addr + (((2 * g) ^ (r & 7)) << 4));
-          const uint4 xb = ld_shared_v4(row_addr + (((2 * g + 1) ^ (r & 7)) << 4));
-          const uint4 sa = ld_shared_v4(s_sm(s, c) + g * 32);
-          const uint4 sb = ld_shared_v4(s_sm(s, c) + g * 32 + 16);
-          const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      const int kc = c_begin + 2 * i + c;         // this thread's chunk of 64 k
+      // In a range's last stage the second chunk may be absent: those lanes
+      // compute nothing but still take part in the shuffles below.
+      const bool active = kc < c_end;
+      uint32_t sca = 0, scb = 0;
+      if (active) {
+        uint64_t nsm[8];
+        {
+          const uint4 sa = lds_v4(s_sm(s) + cg * 32);
+          const uint4 sb = lds_v4(s_sm(s) + cg * 32 + 16);
           const uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-          const uint64_t codes = quantize_group(xw, sw, scale);
-          if (row < p.M) {
-            uint2* dst = reinterpret_cast<uint2*>(p.qact + static_cast<size_t>(row) * half_k +
-                                                  kc * (BKE / 2) + g * 8);
-            *dst = make_uint2(static_cast<uint32_t>(codes), static_cast<uint32_t>(codes >> 32));
-          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) nsm[j] = bf16x2_to_pk(sw[j] ^ 0x80008000u);
         }
-        // Tiled scales: 512-byte block per (128 rows, 4 groups); byte
-        // (row % 32) * 16 + ((row % 128) / 32) * 4 + g.  Lanes 4j..4j+3 hold
-        // one row's four groups of one chunk; every lane takes part in the
-        // shuffles.
-        uint32_t w = scale << (8 * g);
-        w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
-        w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
-        if (active && g == 0 && row < rows_pad) {
-          uint32_t* sdst = reinterpret_cast<uint32_t*>(
-              p.ascales_tiled + (static_cast<size_t>(row >> 7) * p.chunks + kc) * 512 +
-              (row & 31) * 16 + ((row & 127) >> 5) * 4);
-          *sdst = w;
-        }
+        const uint32_t xs = s_x(s);
+        const uint4 a0 = lds_v4(xs + xo0), a1 = lds_v4(xs + xo1);
+        const uint4 b0 = lds_v4(xs + xo0 + 64 * 128), b1 = lds_v4(xs + xo1 + 64 * 128);
+        const uint32_t xa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const uint32_t xb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const uint64_t ca = quantize_group(xa, nsm, sca);
+        const uint64_t cb = quantize_group(xb, nsm, scb);
+        if (m0 < p.M)
+          *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
+              make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
+        if (m1 < p.M)
+          *reinterpret_cast<uint2*>(q1_row + kc * (BKE / 2)) =
+              make_uint2(static_cast<uint32_t>(cb), static_cast<uint32_t>(cb >> 32));
+      }
+      // Lanes 4j..4j+3 hold one row's four groups of one chunk.
+      uint32_t wa = sca << (8 * g), wb = scb << (8 * g);
+      wa |= __shfl_xor_sync(0xFFFFFFFFu, wa, 1);
+      wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 1);
+      wa |= __shfl_xor_sync(0xFFFFFFFFu, wa, 2);
+      wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 2);
+      if (active && g == 0) {
+        uint8_t* blk = sc_base + static_cast<size_t>(kc) * 512;
+        *reinterpret_cast<uint32_t*>(blk + sc_off0) = wa;
+        *reinterpret_cast<uint32_t*>(blk + sc_off1) = wb;
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
     }
-    if (ok) l_ready = __all_sync(0xFFFFFFFFu, svdq_wait(lfull_bar, 0, SITE_LFULL));
-  }
+    const bool l_ready = ok && __all_sync(0xFFFFFFFFu, svdq_wait(lfull_bar, 0, SITE_LFULL));
 
-  // --------------------------------------------------- low-rank readout --
-  // TMEM holds L^T: lane r, column m.  The four quantizer warps of lane
-  // quarter (w % 4) read its columns in four slices of bm / 4.
-  const bool is_q = warp >= 2;
-  const int lq = warp & 3;
-  const int slice = (warp - 2) >> 2;
-  const int r_lane = lq * 32 + lane;
-  const int cw = bm >> 2;  // columns per warp (multiple of 8)
-  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lq * 32) << 16);
-  if (p.split == 1) {
-    if (is_q && l_ready) {
+    // ------------------------------------------------- low-rank readout --
+    // TMEM holds L^T: lane r, column m.  The four quantizer warps of lane
+    // quarter (warp % 4) read 32 columns each.
+    const int lq = warp & 3;
+    const int slice = (warp - 2) >> 2;
+    const int r = lq * 32 + lane;
+    const int mc = slice * 32;
+    uint32_t v[32];
+    if (l_ready) {
       tc_fence_after();
-      for (int c0 = slice * cw; c0 < (slice + 1) * cw; c0 += 8) {
-        uint32_t v[8];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-              "=r"(v[6]), "=r"(v[7])
-            : "r"(lane_addr + c0)
-            : "memory");
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int row = mb * bm + c0 + j;
-          if (row < p.M)
-            p.lowrank[static_cast<size_t>(row) * R + r_lane] =
-                __float2bfloat16_rn(__uint_as_float(v[j]));
-        }
-      }
+      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(lq * 32) << 16) + mc, v);
+      tmem_ld_wait();
     }
-  } else {
-    // Partial sums: every quantizer warp has finished with the ring before
-    // any of them overwrites it with its fp32 partial (row-major [m][r]).
-    if (is_q) {
-      named_bar_sync(1, NUM_QTHREADS);
+    if (p.split == 1) {
       if (l_ready) {
-        tc_fence_after();
-        for (int c0 = slice * cw; c0 < (slice + 1) * cw; c0 += 8) {
-          uint32_t v[8];
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-                "=r"(v[6]), "=r"(v[7])
-              : "r"(lane_addr + c0)
-              : "memory");
-          tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            st_shared_f32(s_ring + ((c0 + j) * PART_STRIDE + r_lane) * 4, __uint_as_float(v[j]));
+        for (int j = 0; j < 32; ++j) {
+          const int m = mb * BM + mc + j;
+          if (m < p.M)
+            p.lowrank[static_cast<size_t>(m) * R + r] = __float2bfloat16_rn(__uint_as_float(v[j]));
         }
       }
-    }
-    __syncwarp();
-    cluster_sync_all();
-    if (is_q && !error_raised()) {
-      // This rank sums its share of the bm x 32 float4 units over all ranks.
-      const int units = bm * (R / 4);
-      const int u0 = rank * units / p.split;
-      const int u1 = (rank + 1) * units / p.split;
-      for (int u = u0 + (threadIdx.x - 64); u < u1; u += NUM_QTHREADS) {
-        const int m = u / (R / 4);
-        const int c4 = u % (R / 4);
-        const uint32_t off = s_ring + (m * PART_STRIDE + 4 * c4) * 4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      // fp32 partial [m][r] of this K range, then count this CTA in.
+      float* part = p.partials + (static_cast<size_t>(ks) * p.m_tiles + mb) * (BM * R);
+      if (l_ready) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) part[(mc + j) * R + r] = __uint_as_float(v[j]);
+      }
+      __threadfence();
+      named_bar_sync(1, NUM_QTHREADS);
+      if (qt == 0) {
+        // Count only a CTA whose partial is complete; a failed CTA leaves
+        // the tile unfinished (and its counter for the caller to reset).
+        const uint32_t old = l_ready ? atomicAdd(p.counters + mb, 1u) : 0xFFFFFFFFu;
+        *flag_ptr = (old == static_cast<uint32_t>(p.split - 1)) ? 1u : 0u;
+      }
+      named_bar_sync(1, NUM_QTHREADS);
+      if (*flag_ptr != 0u) {
+        __threadfence();
+        // Last CTA of the tile: L = sum over K ranges in order, to bf16.
+        float acc[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
         for (int src = 0; src < p.split; ++src) {
-          const float4 t = ld_dsmem_f4(map_to_rank(off, src));
-          acc.x += t.x;
-          acc.y += t.y;
-          acc.z += t.z;
-          acc.w += t.w;
+          const float* sp = p.partials + (static_cast<size_t>(src) * p.m_tiles + mb) * (BM * R);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[j] += __ldcg(sp + (mc + j) * R + r);
         }
-        const int row = mb * bm + m;
-        if (row < p.M) {
-          __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-          __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-          uint2* dst = reinterpret_cast<uint2*>(p.lowrank + static_cast<size_t>(row) * R + 4 * c4);
-          *dst = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int m = mb * BM + mc + j;
+          if (m < p.M) p.lowrank[static_cast<size_t>(m) * R + r] = __float2bfloat16_rn(acc[j]);
         }
+        if (qt == 0) p.counters[mb] = 0u;
       }
     }
-    __syncwarp();
-    cluster_sync_all();
   }
 
   // ----------------------------------------------------------- teardown --
@@ -477,7 +431,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x [M, ldx] b
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, ncols);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
