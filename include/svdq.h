@@ -26,9 +26,9 @@
  *   last index contiguous.
  * - Memory: every tensor pointer is a DEVICE pointer on the current CUDA
  *   device, unless a parameter says otherwise.  The caller owns and
- *   allocates every buffer, workspaces included (sizes from the
- *   svdq_*_bytes queries); the library allocates nothing apart from a few
- *   static device words (an error word and a counter).
+ *   allocates every buffer (sizes from the svdq_*_bytes queries); the
+ *   library allocates nothing apart from a few static device words (an
+ *   error word and a counter).
  * - Streams: `stream` is a cudaStream_t passed as void* (NULL = the
  *   legacy default stream).  Calls only enqueue work and return; nothing
  *   synchronizes the host except where a call says so.
@@ -67,7 +67,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 3
+#define SVDQ_ABI_VERSION 4
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -85,13 +85,6 @@ size_t svdq_wscales_tiled_bytes(int N, int K);
 /* Low-rank activations L = x @ proj_down written by svdq_quantize_act:
  * M * R bf16 values ([M, R] row-major). */
 size_t svdq_lowrank_bytes(int M, int R);
-
-/* Workspace svdq_quantize_act needs for an [M, K] input on the current
- * device: 0 when the K dimension is not split (large M), else a 4096-byte
- * counter area (one 32-bit counter per 128-row tile) followed by
- * split * ceil(M/128) * 64 KB of fp32 partial low-rank tiles.  Needs a
- * device; 0 on bad arguments or without a usable device. */
-size_t svdq_quantize_workspace_bytes(int M, int K);
 
 /* ---- the path ---------------------------------------------------------- */
 
@@ -111,9 +104,10 @@ int svdq_repack_weights(const uint8_t* wscales, int N, int K,
 
 /* Activation side of the layer (model card runtime formula): reads x once
  * and writes quant(x * smooth) and the low-rank product x @ proj_down.
- * The work is cut into 128-row tiles and, for small M, `split` K ranges
- * per tile (svdq_quantize_plan); the K ranges' fp32 partial products of
- * L are summed in K-range order, so results do not depend on timing.
+ * The work is cut into tiles of 64 or 128 rows and, for small M, `split`
+ * K ranges per tile handled by a thread-block cluster
+ * (svdq_quantize_plan); the K ranges' fp32 partial products of L are
+ * summed in K-range order on chip, so results do not depend on timing.
  *   x           [M, ldx] bf16, first K columns used; ldx >= K, ldx % 8 == 0.
  *   smooth      [K] bf16 smoothing factor (multiplied, not divided).
  *   proj_down   [K, R] bf16.
@@ -125,22 +119,11 @@ int svdq_repack_weights(const uint8_t* wscales, int N, int K,
  *               Read its logical [M, K/16] form with svdq_unpack_scales.
  *   lowrank     out, [M, R] bf16: x @ proj_down accumulated in fp32 and
  *               rounded to bf16 (the raw x, not x * smooth).
- *   workspace   device scratch of workspace_bytes >=
- *               svdq_quantize_workspace_bytes(M, K) bytes, 256-byte
- *               aligned; may be NULL when that size is 0 (else
- *               SVDQ_ERR_INVALID_ARG).  Its first 4096 bytes (the
- *               counters) must be zero before the first call: zero the
- *               buffer once after allocating it.  Every call that
- *               completes leaves them zero again, whatever its shape;
- *               after a call that reported an error, zero them before
- *               reusing the buffer.  Calls that share a workspace must not
- *               overlap on the GPU (use one stream, or one workspace per
- *               stream).
  * Limits: K % 64 == 0 (else SVDQ_ERR_UNSUPPORTED). */
 int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx,
                       const uint16_t* smooth, const uint16_t* proj_down, int R,
                       uint8_t* qact, void* ascales_tiled, uint16_t* lowrank,
-                      void* workspace, size_t workspace_bytes, void* stream);
+                      void* stream);
 
 /* Block-scaled FP4 GEMM with the fused epilogue (model card runtime
  * formula):
@@ -166,10 +149,10 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
 /* ---- helpers ------------------------------------------------------------ */
 
 /* Launch shape svdq_quantize_act uses on the current device for an [M, K]
- * input: rows per tile (*bm, 128) and the number of K ranges per tile
- * (*split, 1..16): ceil(M/128) * split CTAs, enough to cover the SMs once
- * when M is small, with at least 256 k per range.  For inspection and
- * tests; needs a device. */
+ * input: rows per tile (*bm, 64 or 128) and the number of K ranges per
+ * tile (*split: 1, 2, 4 or 8 CTAs of a cluster, at least 256 k each),
+ * chosen to occupy the most SMs in one wave.  For inspection and tests;
+ * needs a device. */
 int svdq_quantize_plan(int M, int K, int* bm, int* split);
 
 /* Inverse of the tile order, for tests and inspection: tiled scales of

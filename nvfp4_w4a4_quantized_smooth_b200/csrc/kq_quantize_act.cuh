@@ -29,26 +29,28 @@
 // code must carry.  A scale that rounds to zero gives -r = -0 and therefore
 // signed zero codes.
 //
-// CTA work item: a tile of BM = 128 rows and one of `split` ranges of K.
-// 18 warps:
+// CTA work item: a tile of BM rows (64 or 128, a template parameter) and
+// one of `split` ranges of K; the `split` CTAs of a tile form a
+// thread-block cluster.  18 warps:
 //   warp 0      TMA producer: per stage of 128 k, the x tile (one 3-D box:
-//               2 chunks x [128 rows x 64 k] bf16, 128-byte swizzle), the
+//               2 chunks x [BM rows x 64 k] bf16, 128-byte swizzle), the
 //               proj_down rows (one 3-D box: 2 halves of 64 r x [128 k x
-//               128 B]) and 256 B of smooth, into a ring of 3 stages.
+//               128 B]) and 256 B of smooth, into a ring of stages.
 //   warp 1      TMEM owner, MMA issuer.  The low-rank product is computed
-//               transposed, L^T[128 x 128] += proj_down_stage^T x_tile^T:
-//               tcgen05.mma kind::f16, M = 128 (= R), N = 128 (rows),
-//               K = 16; A (proj_down) MN-major, B (x tile) K-major, fp32
-//               accumulator in 128 TMEM columns.
+//               transposed, L^T[128 x BM] += proj_down_stage^T x_tile^T:
+//               tcgen05.mma kind::f16, M = 128 (= R), N = BM, K = 16;
+//               A (proj_down) MN-major, B (x tile) K-major, fp32
+//               accumulator in BM TMEM columns.
 //   warps 2..17 quantizers: thread t owns 16-element group (t % 8) of the
-//               stage's 128 k and rows t / 8 and t / 8 + 64, so it converts
-//               its 16 smooth values once per stage and runs two
-//               independent groups side by side; writes packed codes and
-//               tiled scales; afterwards reads L^T out of TMEM.
+//               stage's 128 k and row t / 8 (and t / 8 + 64 when BM = 128,
+//               two independent groups side by side); it converts its 16
+//               smooth values once per stage; writes packed codes and tiled
+//               scales; afterwards reads L^T out of TMEM.
 // With split == 1 the tile's L is rounded to bf16 and written directly.
-// Otherwise each CTA writes its fp32 partial to the workspace and counts
-// itself in; the last CTA of a row tile sums the split partials in K order
-// (deterministic), writes bf16 L and resets the tile's counter to zero.
+// Otherwise every rank stages its fp32 partial in its own (idle) stage
+// ring, and after a cluster barrier each rank sums a 1/split slice of the
+// tile over all ranks in rank order (deterministic) through distributed
+// shared memory and writes it as bf16.
 #pragma once
 
 #include <cuda.h>
@@ -61,25 +63,32 @@ namespace svdq {
 namespace kq {
 
 constexpr int R = 128;                 // rank (MMA M)
-constexpr int BM = 128;                // rows per tile (MMA N)
 constexpr int BKE = 64;                // k per chunk (one 128-byte swizzled box row)
 constexpr int STAGE_K = 128;           // k per stage (2 chunks)
-constexpr int STAGES = 3;
-constexpr uint32_t X_CHUNK = BM * 128;             // [128 rows x 64 k] bf16, 16 KB
-constexpr uint32_t X_BYTES = 2 * X_CHUNK;          // 32 KB
 constexpr uint32_t PD_HALF = STAGE_K * 128;        // [128 k x 64 r] bf16, 16 KB
 constexpr uint32_t PD_BYTES = 2 * PD_HALF;         // 32 KB
 constexpr uint32_t SM_BYTES = STAGE_K * 2;         // 256 B
-constexpr uint32_t STAGE_BYTES = (X_BYTES + PD_BYTES + SM_BYTES + 1023u) & ~1023u;
 constexpr int NUM_QWARPS = 16;
 constexpr int NUM_QTHREADS = NUM_QWARPS * 32;
 constexpr int NUM_THREADS = 64 + NUM_QTHREADS;
 constexpr uint32_t BAR_BYTES = 128;
-constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-constexpr uint32_t TMEM_COLS = 128;
-constexpr uint32_t PART_BYTES = BM * R * 4;        // one fp32 partial tile, 64 KB
-constexpr int MAX_SPLIT_TILES = 1024;              // row tiles that may split K
-constexpr uint32_t COUNTER_BYTES = MAX_SPLIT_TILES * 4;   // workspace counter area
+constexpr uint32_t SMEM_BUDGET = 227 * 1024;
+constexpr int PART_STRIDE = R + 4;     // floats per row of a staged partial (bank spread)
+constexpr int MAX_SPLIT = 8;
+
+template <int BM>
+struct Shape {
+  static constexpr uint32_t X_CHUNK = BM * 128;             // [BM rows x 64 k] bf16
+  static constexpr uint32_t X_BYTES = 2 * X_CHUNK;
+  static constexpr uint32_t STAGE_BYTES = (X_BYTES + PD_BYTES + SM_BYTES + 1023u) & ~1023u;
+  static constexpr int STAGES_FIT = static_cast<int>((SMEM_BUDGET - BAR_BYTES - 1024) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT < 4 ? STAGES_FIT : 4;
+  static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = BM;                 // 64 or 128 (powers of 2)
+  static constexpr int ROWS_PER_THREAD = BM / 64;           // 1 or 2
+  static_assert(STAGES >= 3, "at least three stages");
+  static_assert(BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partial fits the ring");
+};
 
 constexpr uint32_t SITE_PROD = 0x20, SITE_MMA = 0x21, SITE_QUANT = 0x22, SITE_LFULL = 0x23;
 
@@ -88,12 +97,9 @@ struct Params {
   uint8_t* qact;
   uint8_t* ascales_tiled;
   __nv_bfloat16* lowrank;
-  float* partials;        // [split][m_tiles][BM][R] fp32 (split > 1)
-  uint32_t* counters;     // [m_tiles], zero between launches (split > 1)
   int M, K;
   int chunks;   // K / 64
-  int split;    // K ranges per row tile
-  int m_tiles;
+  int split;    // K ranges per row tile = cluster size
 };
 
 __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
@@ -175,35 +181,36 @@ __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
   return static_cast<uint64_t>(cvt_e2m1x8(qlo)) | (static_cast<uint64_t>(cvt_e2m1x8(qhi)) << 32);
 }
 
+template <int BM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/64}, box {64, 128, 2}
+quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/64}, box {64, BM, 2}
                     const __grid_constant__ CUtensorMap tm_pd,   // proj_down {64, K, 2}, box {64, 128, 2}
                     const Params p) {
+  using S = Shape<BM>;
+  constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t s_ring = smem_u32(smem);
-  const uint32_t s_bar = s_ring + STAGES * STAGE_BYTES;
-  // Stage layout: x [chunk][128 rows x 128 B], proj_down [r half][128 k x
+  const uint32_t s_bar = s_ring + STAGES * S::STAGE_BYTES;
+  // Stage layout: x [chunk][BM rows x 128 B], proj_down [r half][128 k x
   // 128 B], smooth [128 k] bf16.
-  auto s_x = [&](uint32_t s) { return s_ring + s * STAGE_BYTES; };
-  auto s_pd = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + X_BYTES; };
-  auto s_sm = [&](uint32_t s) { return s_ring + s * STAGE_BYTES + X_BYTES + PD_BYTES; };
+  auto s_x = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES; };
+  auto s_pd = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES; };
+  auto s_sm = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES + PD_BYTES; };
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
   const uint32_t lfull_bar = s_bar + 16u * STAGES;
   const uint32_t final_bar = lfull_bar + 8u;
-  const uint32_t flag_slot = lfull_bar + 16u;
-  const uint32_t tmem_slot = lfull_bar + 20u;
+  const uint32_t tmem_slot = lfull_bar + 16u;
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
-  volatile uint32_t* flag_ptr = reinterpret_cast<volatile uint32_t*>(smem + (flag_slot - s_ring));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int mb = blockIdx.x % p.m_tiles;
-  const int ks = blockIdx.x / p.m_tiles;
-  const int c_begin = ks * p.chunks / p.split;      // in chunks of 64 k
-  const int c_end = (ks + 1) * p.chunks / p.split;
+  const int mb = blockIdx.y;
+  const int rank = blockIdx.x;   // == rank in the cluster (cluster dims = (split, 1, 1))
+  const int c_begin = rank * p.chunks / p.split;      // in chunks of 64 k
+  const int c_end = (rank + 1) * p.chunks / p.split;
   // >= 1 chunk per CTA (host guarantees split <= chunks); the last stage of
   // a range may hold one chunk.
   const int nstages = (c_end - c_begin + 1) / 2;
@@ -220,13 +227,15 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
+
+  bool l_ready = false;   // quantizer threads: L^T accumulator readable
 
   if (warp == 0) {
     if (lane == 0) {
@@ -244,7 +253,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
         const int nc = c_end - kc0 < 2 ? 1 : 2;
         // Boxes are always delivered whole (zero fill past M and K); only
         // the smooth copy is cut to the chunks that exist.
-        mbar_arrive_expect_tx(full_bar(s), X_BYTES + PD_BYTES + nc * 128u);
+        mbar_arrive_expect_tx(full_bar(s), S::X_BYTES + PD_BYTES + nc * 128u);
         tma_load_3d(s_x(s), &tm_x, 0, mb * BM, kc0, full_bar(s));
         tma_load_3d(s_pd(s), &tm_pd, 0, kc0 * BKE, 0, full_bar(s));
         bulk_load(s_sm(s), p.smooth + kc0 * BKE, nc * 128u, full_bar(s));
@@ -278,7 +287,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
         for (int kk = 0; kk < nk; ++kk) {
           mma_f16(tmem_base,
                   smem_desc(s_pd(s) + 2048 * kk, PD_HALF, 1024, kLayoutSwizzle128B),
-                  smem_desc(s_x(s) + (kk >> 2) * X_CHUNK + 32 * (kk & 3), 16, 1024,
+                  smem_desc(s_x(s) + (kk >> 2) * S::X_CHUNK + 32 * (kk & 3), 16, 1024,
                             kLayoutSwizzle128B),
                   idesc, (i | kk) != 0 ? 1u : 0u);
         }
@@ -294,22 +303,25 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
     const int cg = qt & 7;          // group of 16 within the stage's 128 k
     const int c = cg >> 2;          // chunk
     const int g = cg & 3;           // group within the chunk
-    const int r0 = qt >> 3;         // rows r0 and r0 + 64 of the tile
+    const int r0 = qt >> 3;         // row r0 (and r0 + 64) of the tile
     const int half_k = p.K / 2;
     // swizzled 16-byte x chunk positions of this group (same for both rows)
     const uint32_t xo0 =
-        static_cast<uint32_t>(c) * X_CHUNK + r0 * 128 + ((((2 * g) ^ r0) & 7) << 4);
+        static_cast<uint32_t>(c) * S::X_CHUNK + r0 * 128 + ((((2 * g) ^ r0) & 7) << 4);
     const uint32_t xo1 =
-        static_cast<uint32_t>(c) * X_CHUNK + r0 * 128 + ((((2 * g + 1) ^ r0) & 7) << 4);
+        static_cast<uint32_t>(c) * S::X_CHUNK + r0 * 128 + ((((2 * g + 1) ^ r0) & 7) << 4);
     const int m0 = mb * BM + r0;
     const int m1 = m0 + 64;
     uint8_t* q0_row = p.qact + static_cast<size_t>(m0) * half_k + g * 8;
     uint8_t* q1_row = p.qact + static_cast<size_t>(m1) * half_k + g * 8;
     // tiled scales: 512-byte block per (128 rows, 64 k); byte
     // (row % 32) * 16 + ((row % 128) / 32) * 4 + group
-    uint8_t* sc_base = p.ascales_tiled + static_cast<size_t>(mb) * p.chunks * 512;
-    const uint32_t sc_off0 = (r0 & 31) * 16 + (r0 >> 5) * 4;
-    const uint32_t sc_off1 = (r0 & 31) * 16 + ((r0 + 64) >> 5) * 4;
+    uint8_t* sc0 = p.ascales_tiled + static_cast<size_t>(m0 >> 7) * p.chunks * 512 +
+                   (m0 & 31) * 16 + ((m0 & 127) >> 5) * 4;
+    uint8_t* sc1 = p.ascales_tiled + static_cast<size_t>(m1 >> 7) * p.chunks * 512 +
+                   (m1 & 31) * 16 + ((m1 & 127) >> 5) * 4;
+    // rows the tiled scale buffer holds (M rounded up to 128)
+    const int rows_pad = (p.M + 127) & ~127;
     bool ok = true;
     for (int i = 0; i < nstages; ++i) {
       const uint32_t s = static_cast<uint32_t>(i) % STAGES;
@@ -334,92 +346,129 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
         }
         const uint32_t xs = s_x(s);
         const uint4 a0 = lds_v4(xs + xo0), a1 = lds_v4(xs + xo1);
-        const uint4 b0 = lds_v4(xs + xo0 + 64 * 128), b1 = lds_v4(xs + xo1 + 64 * 128);
         const uint32_t xa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const uint32_t xb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        const uint64_t ca = quantize_group(xa, nsm, sca);
-        const uint64_t cb = quantize_group(xb, nsm, scb);
-        if (m0 < p.M)
-          *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
-              make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
-        if (m1 < p.M)
-          *reinterpret_cast<uint2*>(q1_row + kc * (BKE / 2)) =
-              make_uint2(static_cast<uint32_t>(cb), static_cast<uint32_t>(cb >> 32));
+        if constexpr (S::ROWS_PER_THREAD == 2) {
+          const uint4 b0 = lds_v4(xs + xo0 + 64 * 128), b1 = lds_v4(xs + xo1 + 64 * 128);
+          const uint32_t xb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+          const uint64_t ca = quantize_group(xa, nsm, sca);
+          const uint64_t cb = quantize_group(xb, nsm, scb);
+          if (m0 < p.M)
+            *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
+                make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
+          if (m1 < p.M)
+            *reinterpret_cast<uint2*>(q1_row + kc * (BKE / 2)) =
+                make_uint2(static_cast<uint32_t>(cb), static_cast<uint32_t>(cb >> 32));
+        } else {
+          const uint64_t ca = quantize_group(xa, nsm, sca);
+          if (m0 < p.M)
+            *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
+                make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
+        }
       }
       // Lanes 4j..4j+3 hold one row's four groups of one chunk.
-      uint32_t wa = sca << (8 * g), wb = scb << (8 * g);
+      uint32_t wa = sca << (8 * g);
       wa |= __shfl_xor_sync(0xFFFFFFFFu, wa, 1);
-      wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 1);
       wa |= __shfl_xor_sync(0xFFFFFFFFu, wa, 2);
-      wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 2);
-      if (active && g == 0) {
-        uint8_t* blk = sc_base + static_cast<size_t>(kc) * 512;
-        *reinterpret_cast<uint32_t*>(blk + sc_off0) = wa;
-        *reinterpret_cast<uint32_t*>(blk + sc_off1) = wb;
+      if (active && g == 0 && m0 < rows_pad)
+        *reinterpret_cast<uint32_t*>(sc0 + static_cast<size_t>(kc) * 512) = wa;
+      if constexpr (S::ROWS_PER_THREAD == 2) {
+        uint32_t wb = scb << (8 * g);
+        wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 1);
+        wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 2);
+        if (active && g == 0 && m1 < rows_pad)
+          *reinterpret_cast<uint32_t*>(sc1 + static_cast<size_t>(kc) * 512) = wb;
+      } else {
+        // 64-row tiles may end half way through the last 128-row scale
+        // block: the last tile also writes the zero scales of the rows
+        // below it that the block holds.
+        if (active && g == 0 && m1 >= static_cast<int>(gridDim.y) * BM && m1 < rows_pad)
+          *reinterpret_cast<uint32_t*>(sc1 + static_cast<size_t>(kc) * 512) = 0u;
       }
-      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
     }
-    const bool l_ready = ok && __all_sync(0xFFFFFFFFu, svdq_wait(lfull_bar, 0, SITE_LFULL));
+    l_ready = ok && __all_sync(0xFFFFFFFFu, svdq_wait(lfull_bar, 0, SITE_LFULL));
+  }
 
-    // ------------------------------------------------- low-rank readout --
-    // TMEM holds L^T: lane r, column m.  The four quantizer warps of lane
-    // quarter (warp % 4) read 32 columns each.
-    const int lq = warp & 3;
-    const int slice = (warp - 2) >> 2;
-    const int r = lq * 32 + lane;
-    const int mc = slice * 32;
-    uint32_t v[32];
-    if (l_ready) {
+  // ------------------------------------------------- low-rank readout --
+  // TMEM holds L^T: lane r, column m.  The four quantizer warps of lane
+  // quarter (warp % 4) read BM / 4 columns each.
+  const bool is_q = warp >= 2;
+  const int lq = warp & 3;
+  const int slice = (warp - 2) >> 2;
+  const int r = lq * 32 + lane;
+  constexpr int CW = BM / 4;     // 16 or 32 columns per warp
+  const int mc = slice * CW;
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lq * 32) << 16) + mc;
+  if (p.split == 1) {
+    if (is_q && l_ready) {
       tc_fence_after();
-      tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(lq * 32) << 16) + mc, v);
+      uint32_t v[CW];
+      if constexpr (CW == 32) {
+        tmem_ld_32x32b_x32(lane_addr, v);
+      } else {
+        tmem_ld_32x32b_x16(lane_addr, v);
+      }
       tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < CW; ++j) {
+        const int m = mb * BM + mc + j;
+        if (m < p.M) p.lowrank[static_cast<size_t>(m) * R + r] = __float2bfloat16_rn(__uint_as_float(v[j]));
+      }
     }
-    if (p.split == 1) {
+  } else {
+    // Partial sums: every quantizer warp has finished with the ring (and
+    // every MMA has completed) before any of them overwrites it with its
+    // fp32 partial (row-major [m][r], PART_STRIDE floats per row).
+    if (is_q) {
+      named_bar_sync(1, NUM_QTHREADS);
       if (l_ready) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = mb * BM + mc + j;
-          if (m < p.M)
-            p.lowrank[static_cast<size_t>(m) * R + r] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        tc_fence_after();
+        uint32_t v[CW];
+        if constexpr (CW == 32) {
+          tmem_ld_32x32b_x32(lane_addr, v);
+        } else {
+          tmem_ld_32x32b_x16(lane_addr, v);
         }
-      }
-    } else {
-      // fp32 partial [m][r] of this K range, then count this CTA in.
-      float* part = p.partials + (static_cast<size_t>(ks) * p.m_tiles + mb) * (BM * R);
-      if (l_ready) {
+        tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) part[(mc + j) * R + r] = __uint_as_float(v[j]);
+        for (int j = 0; j < CW; ++j)
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(s_ring + ((mc + j) * PART_STRIDE + r) * 4),
+                       "f"(__uint_as_float(v[j]))
+                       : "memory");
       }
-      __threadfence();
-      named_bar_sync(1, NUM_QTHREADS);
-      if (qt == 0) {
-        // Count only a CTA whose partial is complete; a failed CTA leaves
-        // the tile unfinished (and its counter for the caller to reset).
-        const uint32_t old = l_ready ? atomicAdd(p.counters + mb, 1u) : 0xFFFFFFFFu;
-        *flag_ptr = (old == static_cast<uint32_t>(p.split - 1)) ? 1u : 0u;
-      }
-      named_bar_sync(1, NUM_QTHREADS);
-      if (*flag_ptr != 0u) {
-        __threadfence();
-        // Last CTA of the tile: L = sum over K ranges in order, to bf16.
-        float acc[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
+    }
+    __syncwarp();
+    cluster_sync_all();
+    if (is_q && !error_raised()) {
+      // This rank sums its share of the BM x 32 float4 units over all ranks.
+      const int units = BM * (R / 4);
+      const int u0 = rank * units / p.split;
+      const int u1 = (rank + 1) * units / p.split;
+      for (int u = u0 + (threadIdx.x - 64); u < u1; u += NUM_QTHREADS) {
+        const int m = u / (R / 4);
+        const int c4 = u % (R / 4);
+        const uint32_t off = s_ring + (m * PART_STRIDE + 4 * c4) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int src = 0; src < p.split; ++src) {
-          const float* sp = p.partials + (static_cast<size_t>(src) * p.m_tiles + mb) * (BM * R);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) acc[j] += __ldcg(sp + (mc + j) * R + r);
+          const float4 t = ld_dsmem_f4(map_to_rank(off, static_cast<uint32_t>(src)));
+          acc.x += t.x;
+          acc.y += t.y;
+          acc.z += t.z;
+          acc.w += t.w;
         }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int m = mb * BM + mc + j;
-          if (m < p.M) p.lowrank[static_cast<size_t>(m) * R + r] = __float2bfloat16_rn(acc[j]);
+        const int row = mb * BM + m;
+        if (row < p.M) {
+          __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+          uint2* dst = reinterpret_cast<uint2*>(p.lowrank + static_cast<size_t>(row) * R + 4 * c4);
+          *dst = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
         }
-        if (qt == 0) p.counters[mb] = 0u;
       }
     }
+    // No rank leaves while another may still read its shared memory.
+    __syncwarp();
+    cluster_sync_all();
   }
 
   // ----------------------------------------------------------- teardown --
@@ -431,7 +480,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
 }
 

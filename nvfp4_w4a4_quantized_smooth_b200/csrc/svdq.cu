@@ -23,6 +23,9 @@ struct DeviceInfo {
   bool init = false;
   bool sm100 = false;
   int num_sms = 0;
+  // Max co-resident clusters of the activation kernel, by (tile height
+  // 64 / 128, split 1..8); -1 = not queried yet.
+  int kq_clusters[2][svdq::kq::MAX_SPLIT + 1];
 };
 
 std::mutex g_mu;
@@ -47,10 +50,15 @@ int device_setup(DeviceInfo** out) {
       return SVDQ_ERR_CUDA;
     d.sm100 = (major == 10 && minor == 0);
     d.num_sms = sms;
+    for (auto& row : d.kq_clusters)
+      for (int& v : row) v = -1;
     if (d.sm100) {
-      if (cudaFuncSetAttribute(svdq::kq::quantize_act_kernel,
+      if (cudaFuncSetAttribute(svdq::kq::quantize_act_kernel<64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               svdq::kq::SMEM_BYTES) != cudaSuccess ||
+                               svdq::kq::Shape<64>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(svdq::kq::quantize_act_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               svdq::kq::Shape<128>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(svdq::kg::w4a4_linear_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                svdq::kg::SMEM_BYTES) != cudaSuccess)
@@ -118,27 +126,61 @@ int grid_for(size_t work, int threads, int num_sms) {
 }
 
 
-// K ranges per 128-row tile for the activation kernel: enough CTAs to
-// cover the SMs once (one CTA per SM), at most 16, and at least two stages
-// of 128 k per range.
-int kq_split(DeviceInfo* d, int M, int K) {
-  const int m_tiles = (M + svdq::kq::BM - 1) / svdq::kq::BM;
-  if (m_tiles > svdq::kq::MAX_SPLIT_TILES) return 1;
-  const int by_k = K / (2 * svdq::kq::STAGE_K);
-  int split = d->num_sms / m_tiles;
-  if (split > 16) split = 16;
-  if (split > by_k) split = by_k;
-  return split < 1 ? 1 : split;
+// How many clusters of `split` activation-kernel CTAs with tile height
+// `bm` can be resident at once on this device (cached).
+int kq_max_clusters(DeviceInfo* d, int bm, int split) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int& slot = d->kq_clusters[bm == 128 ? 1 : 0][split];
+  if (slot >= 0) return slot;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(split, 1024, 1);
+  cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes =
+      bm == 128 ? svdq::kq::Shape<128>::SMEM_BYTES : svdq::kq::Shape<64>::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const void* fn = bm == 128 ? reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<128>)
+                             : reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<64>);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  slot = n;
+  return n;
 }
 
-// Workspace layout for split > 1: a fixed counter area of
-// svdq::kq::COUNTER_BYTES (one uint32 per row tile, at most 1024 tiles,
-// never written with anything else, so it stays zero between calls of any
-// shape), then the fp32 partial tiles [split][m_tiles][128][128].
-size_t kq_workspace_bytes(int M, int split) {
-  if (split <= 1) return 0;
-  const size_t m_tiles = (M + svdq::kq::BM - 1) / svdq::kq::BM;
-  return svdq::kq::COUNTER_BYTES + static_cast<size_t>(split) * m_tiles * svdq::kq::PART_BYTES;
+// Tile height (64 or 128 rows) and K split (a cluster of 1, 2, 4 or 8
+// CTAs, each with at least two stages of 128 k) of the activation kernel:
+// among the grids that run in one wave (at most one CTA per SM, every
+// cluster co-resident), the one that occupies the most SMs; ties go to the
+// taller tile (less proj_down traffic per row), then to the smaller split.
+// If none fits (very large M), 128-row tiles without a split.
+void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out) {
+  const int chunks = K / svdq::kq::BKE;
+  int best_bm = 128, best_split = 1, best_ctas = -1;
+  for (int bm : {128, 64}) {
+    const int m_tiles = (M + bm - 1) / bm;
+    for (int split = 1; split <= svdq::kq::MAX_SPLIT && (split == 1 || 4 * split <= chunks);
+         split *= 2) {
+      const int ctas = m_tiles * split;
+      if (ctas > d->num_sms) break;
+      if (split > 1 && m_tiles > kq_max_clusters(d, bm, split)) continue;
+      if (ctas > best_ctas) {
+        best_ctas = ctas;
+        best_bm = bm;
+        best_split = split;
+      }
+    }
+  }
+  *bm_out = best_bm;
+  *split_out = best_split;
 }
 }  // namespace
 
@@ -199,39 +241,29 @@ int svdq_repack_weights(const uint8_t* wscales, int N, int K, void* wscales_tile
   return bad ? SVDQ_ERR_INVALID_ARG : SVDQ_OK;
 }
 
-size_t svdq_quantize_workspace_bytes(int M, int K) {
-  if (M < 1 || K < 64 || K % 64) return 0;
-  DeviceInfo* d = nullptr;
-  if (device_setup(&d)) return 0;
-  return kq_workspace_bytes(M, kq_split(d, M, K));
-}
-
 int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* smooth,
                       const uint16_t* proj_down, int R, uint8_t* qact, void* ascales_tiled,
-                      uint16_t* lowrank, void* workspace, size_t workspace_bytes, void* stream) {
+                      uint16_t* lowrank, void* stream) {
   if (!x || !smooth || !proj_down || !qact || !ascales_tiled || !lowrank)
     return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || K < 16 || K % 16 || ldx < K) return SVDQ_ERR_SHAPE;
   if (R != svdq::kq::R || K % 64) return SVDQ_ERR_UNSUPPORTED;
   if (!aligned(x, 16) || !aligned(smooth, 16) || !aligned(proj_down, 16) || !aligned(qact, 16) ||
-      !aligned(ascales_tiled, 16) || !aligned(lowrank, 16) || ldx % 8 ||
-      (workspace && !aligned(workspace, 256)))
+      !aligned(ascales_tiled, 16) || !aligned(lowrank, 16) || ldx % 8)
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
   if (int st = device_setup(&d)) return st;
 
   const int chunks = K / svdq::kq::BKE;
-  const int split = kq_split(d, M, K);
-  const int m_tiles = (M + svdq::kq::BM - 1) / svdq::kq::BM;
-  const size_t need = kq_workspace_bytes(M, split);
-  if (need > 0 && (!workspace || workspace_bytes < need)) return SVDQ_ERR_INVALID_ARG;
+  int bm = 0, split = 0;
+  kq_plan(d, M, K, &bm, &split);
+  const int m_tiles = (M + bm - 1) / bm;
 
   // x viewed as {64 k, M rows, K/64 chunks} and proj_down as {64 r, K,
   // 2 halves of R}, so that one box carries a whole 128-k stage.
   CUtensorMap tm_x, tm_pd;
   if (make_tmap3(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, svdq::kq::BKE, M, chunks,
-                 static_cast<uint64_t>(ldx) * 2, svdq::kq::BKE * 2, svdq::kq::BKE, svdq::kq::BM,
-                 2) ||
+                 static_cast<uint64_t>(ldx) * 2, svdq::kq::BKE * 2, svdq::kq::BKE, bm, 2) ||
       make_tmap3(&tm_pd, proj_down, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, K, 2,
                  static_cast<uint64_t>(R) * 2, 128, 64, svdq::kq::STAGE_K, 2))
     return SVDQ_ERR_CUDA;
@@ -241,17 +273,29 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   p.qact = qact;
   p.ascales_tiled = static_cast<uint8_t*>(ascales_tiled);
   p.lowrank = reinterpret_cast<__nv_bfloat16*>(lowrank);
-  p.counters = static_cast<uint32_t*>(workspace);
-  p.partials = need > 0 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                   svdq::kq::COUNTER_BYTES)
-                        : nullptr;
   p.M = M;
   p.K = K;
   p.chunks = chunks;
   p.split = split;
-  p.m_tiles = m_tiles;
-  svdq::kq::quantize_act_kernel<<<m_tiles * split, svdq::kq::NUM_THREADS, svdq::kq::SMEM_BYTES,
-                                  static_cast<cudaStream_t>(stream)>>>(tm_x, tm_pd, p);
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(split, m_tiles, 1);
+  cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes =
+      bm == 128 ? svdq::kq::Shape<128>::SMEM_BYTES : svdq::kq::Shape<64>::SMEM_BYTES;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e =
+      bm == 128 ? cudaLaunchKernelEx(&cfg, svdq::kq::quantize_act_kernel<128>, tm_x, tm_pd, p)
+                : cudaLaunchKernelEx(&cfg, svdq::kq::quantize_act_kernel<64>, tm_x, tm_pd, p);
+  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
   return launch_status();
 }
 
@@ -311,8 +355,7 @@ int svdq_quantize_plan(int M, int K, int* bm, int* split) {
   if (K % 64) return SVDQ_ERR_UNSUPPORTED;
   DeviceInfo* d = nullptr;
   if (int st = device_setup(&d)) return st;
-  *bm = svdq::kq::BM;
-  *split = kq_split(d, M, K);
+  kq_plan(d, M, K, bm, split);
   return SVDQ_OK;
 }
 

@@ -29,7 +29,7 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 3
+ABI_VERSION = 4
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
 
@@ -44,8 +44,7 @@ SIGNATURES = {
     "svdq_wscales_tiled_bytes": (_SZ, [_I, _I]),
     "svdq_lowrank_bytes": (_SZ, [_I, _I]),
     "svdq_repack_weights": (_I, [_P, _I, _I, _P, _P]),
-    "svdq_quantize_workspace_bytes": (_SZ, [_I, _I]),
-    "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _SZ, _P]),
+    "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
     "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
     "svdq_quantize_plan": (_I, [_I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "svdq_unpack_scales": (_I, [_P, _I, _I, _I, _P, _P]),
@@ -135,45 +134,11 @@ def repack_weights(wscales: torch.Tensor, out: Optional[torch.Tensor] = None,
     return out
 
 
-def quantize_workspace_bytes(M: int, K: int) -> int:
-    """Workspace svdq_quantize_act needs for [M, K] on the current device."""
-    return _lib.svdq_quantize_workspace_bytes(M, K)
-
-
-# One zero-initialised workspace per (device, stream), grown on demand.  The
-# kernel leaves the counter words zero after every call that completes, so
-# a buffer is reused without clearing; calls on one stream never overlap.
-_workspaces = {}
-
-
-def _workspace(nbytes: int, dev: torch.device, stream) -> Optional[torch.Tensor]:
-    if nbytes == 0:
-        return None
-    s = stream if stream is not None else torch.cuda.current_stream(dev)
-    key = (dev.index, s.cuda_stream)
-    ws = _workspaces.get(key)
-    if ws is None or ws.numel() < nbytes:
-        ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
-        _workspaces[key] = ws
-    return ws
-
-
-def reset_workspaces() -> None:
-    """Zero the cached workspaces (needed after a call that reported an error)."""
-    for ws in _workspaces.values():
-        ws.zero_()
-
-
 def quantize_act(x: torch.Tensor, smooth: torch.Tensor, proj_down: torch.Tensor,
                  qact: Optional[torch.Tensor] = None,
                  ascales_tiled: Optional[torch.Tensor] = None,
-                 lowrank: Optional[torch.Tensor] = None, stream=None,
-                 workspace: Optional[torch.Tensor] = None):
-    """x [M, K] bf16 (row stride may exceed K) -> (qact, ascales_tiled, lowrank).
-
-    `workspace`: uint8 device buffer of at least quantize_workspace_bytes(M, K)
-    bytes whose counter words are zero (zero it once after allocating); by
-    default a cached per-stream workspace is used."""
+                 lowrank: Optional[torch.Tensor] = None, stream=None):
+    """x [M, K] bf16 (row stride may exceed K) -> (qact, ascales_tiled, lowrank)."""
     _need(x, torch.bfloat16, "x", 2)
     _need(smooth, torch.bfloat16, "smooth", 1)
     _need(proj_down, torch.bfloat16, "proj_down", 2)
@@ -189,13 +154,9 @@ def quantize_act(x: torch.Tensor, smooth: torch.Tensor, proj_down: torch.Tensor,
                                     device=dev)
     if lowrank is None:
         lowrank = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
-    if workspace is None:
-        workspace = _workspace(quantize_workspace_bytes(M, K), dev, stream)
     _check(_lib.svdq_quantize_act(_ptr(x), M, K, x.stride(0), _ptr(smooth.contiguous()),
                                   _ptr(proj_down.contiguous()), R, _ptr(qact),
-                                  _ptr(ascales_tiled), _ptr(lowrank), _ptr(workspace),
-                                  0 if workspace is None else workspace.numel(),
-                                  _stream(stream)),
+                                  _ptr(ascales_tiled), _ptr(lowrank), _stream(stream)),
            "svdq_quantize_act")
     return qact, ascales_tiled, lowrank
 

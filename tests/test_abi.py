@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(svdq):
 
 
 def test_abi_version_and_status_strings(svdq):
-    assert svdq.abi_version() == 3 == svdq.ABI_VERSION
+    assert svdq.abi_version() == 4 == svdq.ABI_VERSION
     for st in range(8):
         s = svdq._lib.svdq_status_string(st).decode()
         assert s.startswith("SVDQ")
@@ -70,24 +70,24 @@ def test_argument_checks_fail_before_any_device_work(svdq):
     fake = P(0x1000)            # never dereferenced: checks fail first
     # null pointers
     assert lib.svdq_quantize_act(None, 16, 64, 64, fake, fake, 128, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_INVALID_ARG
+                                 None) == svdq.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 64,
                                 256, 128, None, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_repack_weights(None, 64, 64, fake, None) == svdq.SVDQ_ERR_INVALID_ARG
     # shapes
     assert lib.svdq_quantize_act(fake, 0, 64, 64, fake, fake, 128, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_SHAPE
+                                 None) == svdq.SVDQ_ERR_SHAPE
     assert lib.svdq_quantize_act(fake, 16, 40, 40, fake, fake, 128, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_SHAPE
+                                 None) == svdq.SVDQ_ERR_SHAPE
     assert lib.svdq_quantize_act(fake, 16, 64, 32, fake, fake, 128, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_SHAPE
+                                 None) == svdq.SVDQ_ERR_SHAPE
     assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 64,
                                 256, 128, fake, 32, None) == svdq.SVDQ_ERR_SHAPE
     # implemented limits
     assert lib.svdq_quantize_act(fake, 16, 64, 64, fake, fake, 64, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_UNSUPPORTED
+                                 None) == svdq.SVDQ_ERR_UNSUPPORTED
     assert lib.svdq_quantize_act(fake, 16, 80, 80, fake, fake, 128, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_UNSUPPORTED
+                                 None) == svdq.SVDQ_ERR_UNSUPPORTED
     assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 64,
                                 192, 128, fake, 64, None) == svdq.SVDQ_ERR_UNSUPPORTED
     assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 48,
@@ -95,9 +95,9 @@ def test_argument_checks_fail_before_any_device_work(svdq):
     # alignment
     odd = P(0x1001)
     assert lib.svdq_quantize_act(odd, 16, 64, 64, fake, fake, 128, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_ALIGNMENT
+                                 None) == svdq.SVDQ_ERR_ALIGNMENT
     assert lib.svdq_quantize_act(fake, 16, 64, 68, fake, fake, 128, fake, fake, fake,
-                                 None, 0, None) == svdq.SVDQ_ERR_ALIGNMENT
+                                 None) == svdq.SVDQ_ERR_ALIGNMENT
     assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, odd, 16, 64,
                                 256, 128, fake, 64, None) == svdq.SVDQ_ERR_ALIGNMENT
     # scale unpack: only the two documented tile orders
@@ -113,6 +113,5 @@ def test_device_calls_without_a_gpu_report_an_error(svdq):
         pytest.skip("a GPU is present")
     P = ctypes.c_void_p
     fake = P(0x1000)
-    st = svdq._lib.svdq_quantize_act(fake, 16, 64, 64, fake, fake, 128, fake, fake, fake, None, 0,
-                                      None)
+    st = svdq._lib.svdq_quantize_act(fake, 16, 64, 64, fake, fake, 128, fake, fake, fake, None)
     assert st in (svdq.SVDQ_ERR_CUDA, svdq.SVDQ_ERR_ARCH)
