@@ -163,7 +163,11 @@ class ClockSampler:
 
 # -------------------------------------------------------- distributed ----
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """Join the job torchrun started (RANK / WORLD_SIZE / MASTER_* from the
+    environment).  Ranks are independent replicas: the only collectives are
+    the barriers around the timed region and the max of the elapsed times.
+    `gloo` (CPU) serves the host-side tests of this logic."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -171,9 +175,13 @@ def dist_setup():
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout,
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
     return world, rank, local
 
 
@@ -184,13 +192,27 @@ def barrier(world):
 
 
 def max_over_ranks(value, world):
+    """Max of a per-rank float over all ranks (every rank gets it)."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(workload, rank):
+    """Each rank draws its own token batch (weak scaling: independent
+    problems of the same shape on every GPU)."""
+    from nvfp4_w4a4_quantized_smooth_b200 import synth
+    return synth.workload_seed(workload) + 7919 * rank
+
+
+def job_value(flops_one_step, steps, world, elapsed_ms):
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's time."""
+    return flops_one_step * steps * world / (elapsed_ms * 1e-3) / 1e12
 
 
 # ------------------------------------------------------ our CUDA path ----
@@ -244,7 +266,7 @@ def bench_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     M, K, N = synth.WORKLOADS[args.workload]
-    seed = synth.workload_seed(args.workload) + 7919 * rank
+    seed = rank_seed(args.workload, rank)
     one = flops_per_step(M, K, N)
 
     # rotating sets: enough that a set is evicted from L2 before it returns
@@ -285,7 +307,7 @@ def bench_ours(args, world, rank, local):
     kq_avg = sum(kq_ms) / K_steps
     kg_avg = sum(kg_ms) / K_steps
 
-    value = one * K_steps * world / (elapsed_ms * 1e-3) / 1e12
+    value = job_value(one, K_steps, world, elapsed_ms)
     peaks, peak_src = load_peaks()
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     hbm = peaks["hbm_gbs"]
@@ -373,7 +395,7 @@ def bench_e2e(args, svdq, d, dev, M, K, N, world):
         torch.cuda.synchronize(dev)
         barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world)
-    val = flops_per_step(M, K, N) * steps * world / (ms * 1e-3) / 1e12
+    val = job_value(flops_per_step(M, K, N), steps, world, ms)
     return {"value": round(val, 2), "unit": UNIT,
             "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
             "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}

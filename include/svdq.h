@@ -37,8 +37,11 @@
  *   check returns its status and enqueues nothing.  A launch failure
  *   returns SVDQ_ERR_CUDA.  Every wait inside the kernels is bounded;
  *   a kernel that gives up records it in a device error word and returns,
- *   and svdq_check_device_error reports it as SVDQ_ERR_TIMEOUT.  A
- *   recorded error makes later kernels return early until it is read.
+ *   and svdq_check_device_error reports it as SVDQ_ERR_TIMEOUT.  While an
+ *   error is recorded, the waits of later kernels give up at once, so those
+ *   kernels stop at their first wait that is not already complete and their
+ *   outputs are undefined until svdq_check_device_error has read and
+ *   cleared the word.
  * - Device: the calls run only on compute capability 10.0 (B200, sm_100a);
  *   anything else gives SVDQ_ERR_ARCH.
  */
@@ -67,7 +70,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 4
+#define SVDQ_ABI_VERSION 5
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -180,6 +183,15 @@ int svdq_check_device_error(void* stream);
  * of GPU time, for the current device (default 2e9 = 2 s).  0 restores the
  * default.  A short limit is how tests make a wait run out on purpose. */
 int svdq_set_wait_timeout_ns(uint64_t ns);
+
+/* Diagnostic with no counterpart in the method: one thread waits, through
+ * the same bounded wait the kernels use, on a barrier that completes only
+ * if `arrive` is nonzero.  With arrive = 0 the wait runs out after the
+ * current limit (svdq_set_wait_timeout_ns) and records SVDQ_ERR_TIMEOUT,
+ * which the next svdq_check_device_error returns; the context stays
+ * usable.  Enqueues one kernel on `stream`; returns SVDQ_OK, SVDQ_ERR_ARCH
+ * or SVDQ_ERR_CUDA. */
+int svdq_wait_probe(int arrive, void* stream);
 
 #ifdef __cplusplus
 }

@@ -182,6 +182,20 @@ void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out) {
   *bm_out = best_bm;
   *split_out = best_split;
 }
+// One thread waits, through the same bounded wait the layer's kernels use,
+// on an mbarrier that completes only if `arrive` is set.  With arrive = 0
+// nothing completes it, so the wait runs out after the current limit and
+// records a timeout in the device error word.
+__global__ void wait_probe_kernel(int arrive) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = svdq::smem_u32(&bar);
+  svdq::mbar_init(b, 1);
+  svdq::fence_mbar_init();
+  if (arrive) svdq::mbar_arrive(b);
+  svdq::svdq_wait(b, 0u, 0x01u);
+}
+
 }  // namespace
 
 extern "C" {
@@ -401,6 +415,13 @@ int svdq_check_device_error(void* stream) {
       return SVDQ_ERR_CUDA;
     return SVDQ_ERR_TIMEOUT;
   }
+  return launch_status();
+}
+
+int svdq_wait_probe(int arrive, void* stream) {
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(arrive ? 1 : 0);
   return launch_status();
 }
 

@@ -29,7 +29,7 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 4
+ABI_VERSION = 5
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
 
@@ -51,6 +51,7 @@ SIGNATURES = {
     "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
     "svdq_check_device_error": (_I, [_P]),
     "svdq_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
+    "svdq_wait_probe": (_I, [_I, _P]),
 }
 
 
@@ -227,6 +228,12 @@ def check_device_error(stream=None) -> None:
 
 def set_wait_timeout_ns(ns: int) -> None:
     _check(_lib.svdq_set_wait_timeout_ns(ns), "svdq_set_wait_timeout_ns")
+
+
+def wait_probe(arrive: bool, stream=None) -> None:
+    """Enqueue one bounded wait that completes only if ``arrive``; without
+    it the wait runs out and the next check_device_error raises."""
+    _check(_lib.svdq_wait_probe(1 if arrive else 0, _stream(stream)), "svdq_wait_probe")
 
 
 class PreparedWeights:
