@@ -181,6 +181,9 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
+  // Set-up above overlaps the previous kernel; global memory waits for it.
+  griddep_wait();
+  griddep_launch_dependents();
 
   const int num_k = p.K / BK;                  // K steps per tile
   const int tiles = p.m_tiles * p.n_tiles;

@@ -234,6 +234,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
+  // Set-up above overlaps the previous kernel; global memory waits for it.
+  griddep_wait();
+  griddep_launch_dependents();
 
   bool l_ready = false;   // quantizer threads: L^T accumulator readable
 

@@ -113,6 +113,21 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// ------------------------------------------------- dependent launches --
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel in the stream is still running.  griddep_wait blocks
+// until that kernel has completed and its memory operations are visible;
+// every thread calls it before its first access to global memory.  (No-op
+// for a kernel launched without the attribute.)
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next kernel in the stream begin launching (its blocks run their
+// set-up and then wait in griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- TMA --
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

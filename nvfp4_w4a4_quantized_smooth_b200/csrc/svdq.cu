@@ -299,13 +299,15 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   cfg.dynamicSmemBytes =
       bm == 128 ? svdq::kq::Shape<128>::SMEM_BYTES : svdq::kq::Shape<64>::SMEM_BYTES;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = split;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e =
       bm == 128 ? cudaLaunchKernelEx(&cfg, svdq::kq::quantize_act_kernel<128>, tm_x, tm_pd, p)
                 : cudaLaunchKernelEx(&cfg, svdq::kq::quantize_act_kernel<64>, tm_x, tm_pd, p);
@@ -357,9 +359,20 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   p.n_tiles = (N + svdq::kg::BN - 1) / svdq::kg::BN;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < d->num_sms ? tiles : d->num_sms;
-  svdq::kg::w4a4_linear_kernel<<<grid, svdq::kg::NUM_THREADS, svdq::kg::SMEM_BYTES,
-                                 static_cast<cudaStream_t>(stream)>>>(tm_a, tm_b, tm_l, tm_p, tm_y,
-                                                                      p);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(svdq::kg::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = svdq::kg::SMEM_BYTES;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, svdq::kg::w4a4_linear_kernel, tm_a, tm_b, tm_l, tm_p, tm_y, p) !=
+      cudaSuccess)
+    return SVDQ_ERR_CUDA;
   return launch_status();
 }
 
