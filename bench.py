@@ -443,6 +443,179 @@ def bench_e2e(args, svdq, d, dev, M, K, N, world):
                           "2 device buffers)"}
 
 
+# -------------------------------------------------- the 30-block stack ---
+
+def stack_flops(M=None):
+    from nvfp4_w4a4_quantized_smooth_b200 import synth
+    M = synth.TOKENS if M is None else M
+    return synth.DIT_BLOCKS * sum(flops_per_step(M, K, N) for _, K, N in synth.DIT_BLOCK_LINEARS)
+
+
+def bench_stack(args, world, rank, local):
+    """One step = all 150 linears of the 30-block stack (qkv, out, w1, w3,
+    w2 per block; quantize + GEMM each) back to back in one stream, at
+    M = 4352 tokens.  Block inputs and the w2 inputs (silu(y_w1) * y_w3 of
+    the same block, formed once before timing) are resident; weights
+    (3.2 GB) stream from HBM, so no L2 flush is needed."""
+    import torch
+    from nvfp4_w4a4_quantized_smooth_b200 import build as b
+    if rank == 0:
+        b.build()
+    barrier(world)
+    from nvfp4_w4a4_quantized_smooth_b200 import svdq, synth
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    M = synth.TOKENS
+    host = synth.make_stack(M=M, x_seed_offset=7919 * rank)
+    stream = torch.cuda.Stream(device=dev)
+    order = [name for name, _, _ in synth.DIT_BLOCK_LINEARS]
+    with torch.cuda.stream(stream):
+        blocks = []
+        for layers in host:
+            w = {n: svdq.PreparedWeights(L.qweight.to(dev), L.wscales.to(dev),
+                                         L.wcscales.to(dev), L.wtscale.to(dev),
+                                         L.smooth.to(dev), L.proj_down.to(dev),
+                                         L.proj_up.to(dev), L.bias.to(dev), stream=stream)
+                 for n, L in layers.items()}
+            blocks.append({"w": w, "x": layers["qkv"].x.to(dev)})
+        del host
+        # work buffers, one per K (activation side) and per linear (outputs)
+        act = {}
+        for K in {k for _, k, _ in synth.DIT_BLOCK_LINEARS}:
+            act[K] = (torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+                      torch.empty(svdq.ascales_tiled_bytes(M, K), dtype=torch.uint8, device=dev),
+                      torch.empty(M, R, dtype=torch.bfloat16, device=dev))
+        ybuf = {n: torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                for n, _, N in synth.DIT_BLOCK_LINEARS}
+
+        def linear(x, w, y):
+            qa, asc, lr = act[w.K]
+            svdq.quantize_act(x, w.smooth, w.proj_down, qact=qa, ascales_tiled=asc, lowrank=lr,
+                              stream=stream)
+            svdq.w4a4_linear(qa, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
+                             w.proj_up, w.bias, y=y, stream=stream)
+
+        for blk in blocks:   # the w2 inputs, from the GPU's own outputs
+            linear(blk["x"], blk["w"]["w1"], ybuf["w1"])
+            linear(blk["x"], blk["w"]["w3"], ybuf["w3"])
+            blk["h"] = svdq.silu_mul(ybuf["w1"], ybuf["w3"], stream=stream)
+
+        def step(evs=None):
+            j = 0
+            for blk in blocks:
+                for n in order:
+                    x = blk["h"] if n == "w2" else blk["x"]
+                    if evs is not None:
+                        evs[j].record(stream)
+                    linear(x, blk["w"][n], ybuf[n])
+                    j += 1
+            if evs is not None:
+                evs[j].record(stream)
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        svdq.check_device_error(stream)
+        steps = args.steps
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                              int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+        clocks.start()
+        time.sleep(0.2)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for _ in range(steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        # per-linear durations, one more pass with an event between linears
+        n_lin = len(blocks) * len(order)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_lin + 1)]
+        step(evs)
+        torch.cuda.synchronize(dev)
+        clocks.stop()
+        svdq.check_device_error(stream)
+
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
+    flops = stack_flops(M)
+    value = job_value(flops, steps, world, elapsed_ms)
+    per_name = {n: 0.0 for n in order}
+    for j in range(n_lin):
+        per_name[order[j % len(order)]] += evs[j].elapsed_time(evs[j + 1])
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    per_linear = {}
+    for n, K, N in synth.DIT_BLOCK_LINEARS:
+        ms = per_name[n] / len(blocks)
+        per_linear[n] = {"K": K, "N": N, "avg_ms": round(ms, 5),
+                         "TFLOP/s": round(flops_per_step(M, K, N) / (ms * 1e-3) / 1e12, 1)}
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(elapsed_ms / steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3 block16, fp32 accumulate) + bf16 low-rank",
+        "data": "synthetic (seeded; random weights of the stack's shapes)",
+        "config": {"workload": args.workload, "M": M, "blocks": len(blocks),
+                   "linears_per_step": n_lin, "R": R,
+                   "parallelism": f"dp{world} (independent token batches per GPU)",
+                   "l2": "weights of 150 linears (3.2 GB) stream from HBM every step",
+                   "per_linear": per_linear},
+        "roofline": {"bound": "tensor", "kernel": "whole step (150 x quantize + GEMM)",
+                     "achieved": round(value / world, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(value / world / fp4_peak, 4),
+                     "traffic": None,
+                     "peak_source": f"{peak_src} bf16 sustained x {FP4_OVER_BF16:g} (nominal "
+                                    "FP4:BF16 dense ratio; a step of ~16 ms is a sustained load)"},
+        "e2e": None,
+        "gpu_launches": 2 * n_lin * steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_stack(sample_rows=16)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def _stack_oracle_args(rows):
+    """Oracle arguments for `rows` tokens through each linear of block 0 (the
+    w2 input is a seeded plain N(0, 1) stand-in for silu(y_w1) * y_w3)."""
+    import torch
+    from nvfp4_w4a4_quantized_smooth_b200 import synth
+    b = synth.bits
+    layers = synth.make_stack(blocks=1, M=rows)[0]
+    h = synth.make_x(rows, synth.FFN, torch.Generator().manual_seed(4005), outliers=0)
+    args = []
+    for n, L in layers.items():
+        x = h if n == "w2" else L.x
+        args.append((b(x), b(L.smooth), b(L.proj_down), b(L.qweight), b(L.wscales),
+                     b(L.wcscales), b(L.wtscale), b(L.proj_up), b(L.bias)))
+    return args, sum(flops_per_step(rows, K, N) for _, K, N in synth.DIT_BLOCK_LINEARS)
+
+
+def cpu_baseline_stack(sample_rows=16, min_seconds=10.0):
+    """The oracle on a bounded sample of the stack: `sample_rows` tokens
+    through each of the five linear shapes of block 0, repeated until
+    `min_seconds` of CPU work."""
+    from oracle import svdq_ref as ref
+    args, fl = _stack_oracle_args(sample_rows)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        for a in args:
+            ref.svdq_linear_from_x(*a)
+        reps += 1
+        if time.perf_counter() - t0 >= min_seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(fl * reps / dt / 1e12, 6), "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"{sample_rows} tokens through the 5 linears of one block, {reps} passes, "
+                      f"{dt:.1f} s"}
+
+
 # ------------------------------------------------------- the oracle ------
 
 def cpu_baseline(workload, sample_rows=256, min_seconds=10.0):
@@ -488,6 +661,9 @@ def bench_reference(args, world, rank):
         return
     from nvfp4_w4a4_quantized_smooth_b200 import synth
     from oracle import svdq_ref as ref
+    if args.workload == synth.DIT_STACK:
+        bench_reference_stack(args, world)
+        return
     M, K, N = synth.WORKLOADS[args.workload]
     rows = min(32, M)
     L = synth.make_layer(rows, K, N, seed=synth.workload_seed(args.workload))
@@ -517,6 +693,37 @@ def bench_reference(args, world, rank):
     print(json.dumps(out), flush=True)
 
 
+def bench_reference_stack(args, world):
+    """Reference arm on the stack: each step pushes 16 tokens through the
+    five linears of block 0 with the oracle."""
+    from oracle import svdq_ref as ref
+    from nvfp4_w4a4_quantized_smooth_b200 import synth
+    oargs, fl = _stack_oracle_args(16)
+    for a in oargs:
+        ref.svdq_linear_from_x(*a)
+    steps = max(1, min(args.steps, 10))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        for a in oargs:
+            ref.svdq_linear_from_x(*a)
+    dt = time.perf_counter() - t0
+    value = fl * steps / dt / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": 1, "ms_per_step": round(1e3 * dt / steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
+        "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "M": synth.TOKENS, "blocks": synth.DIT_BLOCKS,
+                   "R": R},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _blas_threads(),
+                         "kind": "oracle",
+                         "sample": "each step: 16 tokens through the 5 linears of one block"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -526,7 +733,11 @@ def main(argv=None):
         return
     world, rank, local = dist_setup()
     try:
-        bench_ours(args, world, rank, local)
+        from nvfp4_w4a4_quantized_smooth_b200 import synth
+        if args.workload == synth.DIT_STACK:
+            bench_stack(args, world, rank, local)
+        else:
+            bench_ours(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -35,7 +35,7 @@ R_DEFAULT = 128
 @dataclass
 class LayerOperands:
     """Host (CPU) operands of one layer, in the on-disk layouts."""
-    x: torch.Tensor            # [M, K] bfloat16
+    x: Optional[torch.Tensor]  # [M, K] bfloat16 (None: formed on the device)
     smooth: torch.Tensor       # [K] bfloat16
     qweight: torch.Tensor      # [N, K/2] uint8
     wscales: torch.Tensor      # [K/16, N] uint8 (e4m3fn codes)
@@ -51,7 +51,7 @@ class LayerOperands:
 
     @property
     def K(self) -> int:
-        return self.x.shape[1]
+        return self.qweight.shape[1] * 2
 
     @property
     def N(self) -> int:
@@ -71,6 +71,23 @@ def make_x(M: int, K: int, gen: torch.Generator, outliers: int = 4,
     return x.to(torch.bfloat16)
 
 
+def make_weights(K: int, N: int, R: int, gen: torch.Generator, with_bias: bool = True):
+    """One layer's weights, drawn from `gen` in the fixed order of the module
+    docstring: (smooth, qweight, wscales, wcscales, wtscale, proj_down,
+    proj_up, bias)."""
+    smooth = torch.empty(K).uniform_(0.5, 2.0, generator=gen).to(torch.bfloat16)
+    qweight = torch.randint(0, 256, (N, K // 2), generator=gen, dtype=torch.uint8)
+    wscales = (torch.empty(K // 16, N).uniform_(0.25, 2.0, generator=gen)
+               .to(torch.float8_e4m3fn).view(torch.uint8))
+    wcscales = torch.empty(N).uniform_(0.5, 1.5, generator=gen).to(torch.bfloat16)
+    wtscale = torch.tensor([0.01], dtype=torch.float32).to(torch.bfloat16)
+    proj_down = (torch.randn(K, R, generator=gen) * 0.02).to(torch.bfloat16)
+    proj_up = (torch.randn(N, R, generator=gen) * 0.02).to(torch.bfloat16)
+    bias = ((torch.randn(N, generator=gen) * 0.1).to(torch.bfloat16)
+            if with_bias else None)
+    return smooth, qweight, wscales, wcscales, wtscale, proj_down, proj_up, bias
+
+
 def make_layer(M: int, K: int, N: int, R: int = R_DEFAULT, seed: int = 0,
                outliers: int = 4, outlier_scale: float = 20.0,
                with_bias: bool = True) -> LayerOperands:
@@ -79,18 +96,7 @@ def make_layer(M: int, K: int, N: int, R: int = R_DEFAULT, seed: int = 0,
         raise ValueError("K must be a positive multiple of 16")
     g = torch.Generator().manual_seed(int(seed))
     x = make_x(M, K, g, outliers, outlier_scale)
-    smooth = torch.empty(K).uniform_(0.5, 2.0, generator=g).to(torch.bfloat16)
-    qweight = torch.randint(0, 256, (N, K // 2), generator=g, dtype=torch.uint8)
-    wscales = (torch.empty(K // 16, N).uniform_(0.25, 2.0, generator=g)
-               .to(torch.float8_e4m3fn).view(torch.uint8))
-    wcscales = torch.empty(N).uniform_(0.5, 1.5, generator=g).to(torch.bfloat16)
-    wtscale = torch.tensor([0.01], dtype=torch.float32).to(torch.bfloat16)
-    proj_down = (torch.randn(K, R, generator=g) * 0.02).to(torch.bfloat16)
-    proj_up = (torch.randn(N, R, generator=g) * 0.02).to(torch.bfloat16)
-    bias = ((torch.randn(N, generator=g) * 0.1).to(torch.bfloat16)
-            if with_bias else None)
-    return LayerOperands(x, smooth, qweight, wscales, wcscales, wtscale,
-                         proj_down, proj_up, bias)
+    return LayerOperands(x, *make_weights(K, N, R, g, with_bias))
 
 
 # Named workloads: shapes of one Z-Image-class DiT (hidden 3840, FFN 10240,
@@ -120,6 +126,35 @@ DIT_BLOCK_LINEARS = (
     ("w2", FFN, HIDDEN),
 )
 DIT_BLOCKS = 30
+
+
+# The 30-block stack as one workload: every linear of every block, in
+# execution order, at TOKENS tokens.
+DIT_STACK = "dit_stack_m4352_30x5"
+
+
+def make_stack(blocks: int = DIT_BLOCKS, M: int = TOKENS, R: int = R_DEFAULT,
+               x_seed_offset: int = 0):
+    """Operands of the stack: a list over blocks of {linear name:
+    LayerOperands}.  Each block's input is its own seeded plain N(0, 1)
+    x [M, HIDDEN] (no outlier channels), shared by qkv, out, w1 and w3 (the
+    attention and the norms between them are not part of the layer, so the
+    blocks are independent problems of the same shapes).  The w2 operands
+    carry x = None: its input is silu(y_w1) * y_w3 of the same block, formed
+    from the GPU's own outputs.  Seeds: block input 4000 + 100 b + 5; linear
+    i of block b: 4000 + 100 b + 10 i (`x_seed_offset` moves the inputs
+    only, for independent token batches on other ranks)."""
+    out = []
+    for b in range(blocks):
+        base = workload_seed("dit_stack", layer=b)
+        gx = torch.Generator().manual_seed(base + 5 + x_seed_offset)
+        xb = make_x(M, HIDDEN, gx, outliers=0)
+        layers = {}
+        for i, (name, K, N) in enumerate(DIT_BLOCK_LINEARS):
+            g = torch.Generator().manual_seed(base + 10 * i)
+            layers[name] = LayerOperands(xb if name != "w2" else None, *make_weights(K, N, R, g))
+        out.append(layers)
+    return out
 
 
 def workload_seed(name: str, layer: int = 0) -> int:
