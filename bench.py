@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end (host buffer) measurement")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="stack workloads: skip the CUDA-graph replay measurement")
     return ap.parse_args(argv)
 
 
@@ -465,7 +467,7 @@ def bench_stack(args, world, rank, local):
     from nvfp4_w4a4_quantized_smooth_b200 import svdq, synth
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    M = synth.TOKENS
+    M = synth.DIT_STACKS[args.workload]
     host = synth.make_stack(M=M, x_seed_offset=7919 * rank)
     stream = torch.cuda.Stream(device=dev)
     order = [name for name, _, _ in synth.DIT_BLOCK_LINEARS]
@@ -535,8 +537,33 @@ def bench_stack(args, world, rank, local):
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_lin + 1)]
         step(evs)
         torch.cuda.synchronize(dev)
-        clocks.stop()
         svdq.check_device_error(stream)
+        # The same step captured once as a CUDA graph and replayed: the 300
+        # launches cost one graph launch (reported beside the stream number).
+        graph = None
+        if not args.no_graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step()
+            for _ in range(2):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            gs = torch.cuda.Event(enable_timing=True)
+            ge = torch.cuda.Event(enable_timing=True)
+            barrier(world)
+            gs.record(stream)
+            for _ in range(steps):
+                g.replay()
+            ge.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            svdq.check_device_error(stream)
+            gms = max_over_ranks(gs.elapsed_time(ge), world)
+            graph = {"value": round(job_value(stack_flops(M), steps, world, gms), 2),
+                     "unit": UNIT, "ms_per_step": round(gms / steps, 4),
+                     "what": "the step captured once in a CUDA graph, replayed `steps` times"}
+            del g
+        clocks.stop()
 
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
     flops = stack_flops(M)
@@ -559,7 +586,7 @@ def bench_stack(args, world, rank, local):
         "dtype": "nvfp4 (e2m1 x e4m3 block16, fp32 accumulate) + bf16 low-rank",
         "data": "synthetic (seeded; random weights of the stack's shapes)",
         "config": {"workload": args.workload, "M": M, "blocks": len(blocks),
-                   "linears_per_step": n_lin, "R": R,
+                   "linears_per_step": n_lin, "R": R, "cuda_graph": graph,
                    "parallelism": f"dp{world} (independent token batches per GPU)",
                    "l2": "weights of 150 linears (3.2 GB) stream from HBM every step",
                    "per_linear": per_linear},
@@ -661,7 +688,7 @@ def bench_reference(args, world, rank):
         return
     from nvfp4_w4a4_quantized_smooth_b200 import synth
     from oracle import svdq_ref as ref
-    if args.workload == synth.DIT_STACK:
+    if args.workload in synth.DIT_STACKS:
         bench_reference_stack(args, world)
         return
     M, K, N = synth.WORKLOADS[args.workload]
@@ -713,7 +740,7 @@ def bench_reference_stack(args, world):
         "steps": steps, "warmup": 1, "ms_per_step": round(1e3 * dt / steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
         "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": args.workload, "M": synth.TOKENS, "blocks": synth.DIT_BLOCKS,
+        "config": {"workload": args.workload, "M": synth.DIT_STACKS[args.workload], "blocks": synth.DIT_BLOCKS,
                    "R": R},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _blas_threads(),
                          "kind": "oracle",
@@ -734,7 +761,7 @@ def main(argv=None):
     world, rank, local = dist_setup()
     try:
         from nvfp4_w4a4_quantized_smooth_b200 import synth
-        if args.workload == synth.DIT_STACK:
+        if args.workload in synth.DIT_STACKS:
             bench_stack(args, world, rank, local)
         else:
             bench_ours(args, world, rank, local)

@@ -452,13 +452,21 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
         const int m = u / (R / 4);
         const int c4 = u % (R / 4);
         const uint32_t off = s_ring + (m * PART_STRIDE + 4 * c4) * 4;
+        // All ranks' values are requested before the first add (the
+        // remote loads overlap); the sum still runs in rank order.
+        float4 t[MAX_SPLIT];
+#pragma unroll
+        for (int src = 0; src < MAX_SPLIT; ++src)
+          if (src < p.split) t[src] = ld_dsmem_f4(map_to_rank(off, static_cast<uint32_t>(src)));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < p.split; ++src) {
-          const float4 t = ld_dsmem_f4(map_to_rank(off, static_cast<uint32_t>(src)));
-          acc.x += t.x;
-          acc.y += t.y;
-          acc.z += t.z;
-          acc.w += t.w;
+#pragma unroll
+        for (int src = 0; src < MAX_SPLIT; ++src) {
+          if (src < p.split) {
+            acc.x += t[src].x;
+            acc.y += t[src].y;
+            acc.z += t[src].z;
+            acc.w += t[src].w;
+          }
         }
         const int row = mb * BM + m;
         if (row < p.M) {

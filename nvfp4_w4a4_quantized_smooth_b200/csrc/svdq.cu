@@ -160,22 +160,25 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
 // CTAs, each with at least two stages of 128 k) of the activation kernel:
 // among the grids that run in one wave (at most one CTA per SM, every
 // cluster co-resident), the one that occupies the most SMs; ties go to the
-// taller tile (less proj_down traffic per row), then to the smaller split.
+// tile height that pads M the least, then to the taller tile (less
+// proj_down traffic per row), then to the smaller split.
 // If none fits (very large M), 128-row tiles without a split.
 void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out) {
   const int chunks = K / svdq::kq::BKE;
-  int best_bm = 128, best_split = 1, best_ctas = -1;
+  int best_bm = 128, best_split = 1, best_ctas = -1, best_pad = 0;
   for (int bm : {128, 64}) {
     const int m_tiles = (M + bm - 1) / bm;
+    const int pad = m_tiles * bm - M;
     for (int split = 1; split <= svdq::kq::MAX_SPLIT && (split == 1 || 4 * split <= chunks);
          split *= 2) {
       const int ctas = m_tiles * split;
       if (ctas > d->num_sms) break;
       if (split > 1 && m_tiles > kq_max_clusters(d, bm, split)) continue;
-      if (ctas > best_ctas) {
+      if (ctas > best_ctas || (ctas == best_ctas && pad < best_pad)) {
         best_ctas = ctas;
         best_bm = bm;
         best_split = split;
+        best_pad = pad;
       }
     }
   }

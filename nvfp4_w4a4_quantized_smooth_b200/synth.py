@@ -129,8 +129,10 @@ DIT_BLOCKS = 30
 
 
 # The 30-block stack as one workload: every linear of every block, in
-# execution order, at TOKENS tokens.
+# execution order, at TOKENS tokens; and the same stack at 64 tokens, where
+# weight streaming and launch overhead dominate.
 DIT_STACK = "dit_stack_m4352_30x5"
+DIT_STACKS = {DIT_STACK: TOKENS, "dit_stack_m64_30x5": 64}
 
 
 def make_stack(blocks: int = DIT_BLOCKS, M: int = TOKENS, R: int = R_DEFAULT,

@@ -86,6 +86,8 @@ def test_quantize_plans_fit_one_wave():
             assert split in (1, 2, 4, 8) and (split == 1 or 256 * split <= K), (M, K, split)
             if tiles * split > sms:
                 assert split == 1 and bm == 128, (M, K, bm, split)
+            if M <= 64:
+                assert bm == 64, (M, K, bm)       # the tile that pads M least
 
 
 @pytest.mark.parametrize("M,K", [(300, 3840), (4352, 3840), (16, 10240)])
