@@ -58,8 +58,13 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-def flops_per_step(M, K, N):
-    return 2 * M * N * K + 2 * M * R * (K + N)
+def flops_per_step(M, K, N, r=R):
+    return 2 * M * N * K + 2 * M * r * (K + N)
+
+
+def is_plain(workload):
+    """Workloads of the plain NVFP4 layer (no low-rank branch, no smoothing)."""
+    return workload.startswith("nvfp4_")
 
 
 def load_peaks():
@@ -219,7 +224,7 @@ def job_value(flops_one_step, steps, world, elapsed_ms):
 
 # ------------------------------------------------------ our CUDA path ----
 
-def make_sets(M, K, N, nsets, seed, dev):
+def make_sets(M, K, N, nsets, seed, dev, plain=False):
     import torch
     from nvfp4_w4a4_quantized_smooth_b200 import svdq, synth
     sets = []
@@ -233,6 +238,8 @@ def make_sets(M, K, N, nsets, seed, dev):
         d["qact"] = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
         d["asc"] = torch.empty(svdq.ascales_tiled_bytes(M, K), dtype=torch.uint8, device=dev)
         d["lr"] = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
+        if plain:       # R = 0, no smoothing
+            d["smooth"] = d["proj_down"] = d["proj_up"] = d["lr"] = None
         d["y"] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         sets.append(d)
     return sets
@@ -268,14 +275,16 @@ def bench_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     M, K, N = synth.WORKLOADS[args.workload]
+    plain = is_plain(args.workload)
+    r = 0 if plain else R
     seed = rank_seed(args.workload, rank)
-    one = flops_per_step(M, K, N)
+    one = flops_per_step(M, K, N, r)
 
     # rotating sets: enough that a set is evicted from L2 before it returns
-    probe = make_sets(M, K, N, 1, seed, dev)
+    probe = make_sets(M, K, N, 1, seed, dev, plain)
     per_set = set_bytes(probe[0])
     nsets = max(3, -(-3 * L2_BYTES // per_set))
-    sets = probe + make_sets(M, K, N, nsets - 1, seed + 1, dev)
+    sets = probe + make_sets(M, K, N, nsets - 1, seed + 1, dev, plain)
     repack_us = 1e6 * statistics.median(d["repack_s"] for d in sets)
 
     stream = torch.cuda.Stream(device=dev)
@@ -322,10 +331,11 @@ def bench_ours(args, world, rank, local):
     hbm = peaks["hbm_gbs"]
 
     # roofline of the whole step and of each kernel
-    bytes_kq = 2 * M * K + 2 * K + 2 * K * R + M * K // 2 + M * K // 16 + 2 * M * R
-    bytes_kg = (M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + 4 * N + 2 + 2 * M * R
-                + 2 * N * R + 2 * M * N)
-    flops_kg = 2 * M * N * K + 2 * M * R * N
+    sm_bytes = 0 if plain else 2 * K
+    bytes_kq = 2 * M * K + sm_bytes + 2 * K * r + M * K // 2 + M * K // 16 + 2 * M * r
+    bytes_kg = (M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + 4 * N + 2 + 2 * M * r
+                + 2 * N * r + 2 * M * N)
+    flops_kg = 2 * M * N * K + 2 * M * r * N
     t_roof_step = max(one / (fp4_peak * 1e12), (bytes_kq + bytes_kg) / (hbm * 1e9))
     step_s = elapsed_ms * 1e-3 / K_steps
     kg_tflops = flops_kg / (kg_avg * 1e-3) / 1e12
@@ -333,7 +343,7 @@ def bench_ours(args, world, rank, local):
     traffic = load_traffic("w4a4_linear_kernel")
 
     # end to end through the public API with host buffers
-    e2e = None if args.no_e2e else bench_e2e(args, svdq, sets[0], dev, M, K, N, world)
+    e2e = None if args.no_e2e else bench_e2e(args, svdq, sets[0], dev, M, K, N, world, r)
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
@@ -342,7 +352,8 @@ def bench_ours(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "nvfp4 (e2m1 x e4m3 block16, fp32 accumulate) + bf16 low-rank",
         "data": "synthetic (seeded; random weights of the layer's shapes)",
-        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "R": R,
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "R": r,
+                   "smooth": not plain,
                    "parallelism": f"dp{world} (independent token batches per GPU)",
                    "l2": f"inputs larger than L2: {nsets} rotating sets x "
                          f"{per_set / 2**20:.0f} MiB",
@@ -370,12 +381,12 @@ def bench_ours(args, world, rank, local):
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.workload, sample_rows=256)
+        out["cpu_baseline"] = cpu_baseline(args.workload, sample_rows=256 if not plain else 512)
     if rank == 0:
         print(json.dumps(out), flush=True)
 
 
-def bench_e2e(args, svdq, d, dev, M, K, N, world):
+def bench_e2e(args, svdq, d, dev, M, K, N, world, r=R):
     """Same metric through the public API with the input in pinned host
     memory and the output read back to pinned host memory every step.
 
@@ -436,7 +447,7 @@ def bench_e2e(args, svdq, d, dev, M, K, N, world):
     barrier(world)
     svdq.check_device_error(s_cmp)
     ms = max_over_ranks(start.elapsed_time(end), world)
-    val = job_value(flops_per_step(M, K, N), steps, world, ms)
+    val = job_value(flops_per_step(M, K, N, r), steps, world, ms)
     return {"value": round(val, 2), "unit": UNIT,
             "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
             "d2h_bytes_per_step": y_host.numel() * y_host.element_size(),
@@ -653,22 +664,35 @@ def cpu_baseline(workload, sample_rows=256, min_seconds=10.0):
     from oracle import svdq_ref as ref
     M, K, N = synth.WORKLOADS[workload]
     rows = min(sample_rows, M)
-    L = synth.make_layer(rows, K, N, seed=synth.workload_seed(workload))
-    b = synth.bits
-    args = (b(L.x), b(L.smooth), b(L.proj_down), b(L.qweight), b(L.wscales), b(L.wcscales),
-            b(L.wtscale), b(L.proj_up), b(L.bias))
+    plain = is_plain(workload)
+    fn, args = _oracle_call(synth.make_layer(rows, K, N, seed=synth.workload_seed(workload)),
+                            plain)
     reps = 0
     t0 = time.perf_counter()
     while True:
-        ref.svdq_linear_from_x(*args)
+        fn(*args)
         reps += 1
         if time.perf_counter() - t0 >= min_seconds:
             break
     dt = time.perf_counter() - t0
-    value = flops_per_step(rows, K, N) * reps / dt / 1e12
+    value = flops_per_step(rows, K, N, 0 if plain else R) * reps / dt / 1e12
     return {"value": round(value, 6), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
             "sample": f"{rows} of {M} tokens of {workload} (all K, all N), {reps} passes, "
                       f"{dt:.1f} s"}
+
+
+def _oracle_call(L, plain):
+    """(oracle function, its arguments) for one layer's operands: the full
+    layer, or the plain NVFP4 layer (no low-rank branch, no smoothing)."""
+    from nvfp4_w4a4_quantized_smooth_b200 import synth
+    from oracle import svdq_ref as ref
+    b = synth.bits
+    if plain:
+        return ref.plain_linear_from_x, (b(L.x), b(L.qweight), b(L.wscales), b(L.wcscales),
+                                         b(L.wtscale), b(L.bias))
+    return ref.svdq_linear_from_x, (b(L.x), b(L.smooth), b(L.proj_down), b(L.qweight),
+                                    b(L.wscales), b(L.wcscales), b(L.wtscale), b(L.proj_up),
+                                    b(L.bias))
 
 
 def _blas_threads():
@@ -693,25 +717,24 @@ def bench_reference(args, world, rank):
         return
     M, K, N = synth.WORKLOADS[args.workload]
     rows = min(32, M)
-    L = synth.make_layer(rows, K, N, seed=synth.workload_seed(args.workload))
-    b = synth.bits
-    a = (b(L.x), b(L.smooth), b(L.proj_down), b(L.qweight), b(L.wscales), b(L.wcscales),
-         b(L.wtscale), b(L.proj_up), b(L.bias))
+    plain = is_plain(args.workload)
+    fn, a = _oracle_call(synth.make_layer(rows, K, N, seed=synth.workload_seed(args.workload)),
+                         plain)
     for _ in range(min(args.warmup, 1)):
-        ref.svdq_linear_from_x(*a)
+        fn(*a)
     steps = max(1, min(args.steps, 20))
     t0 = time.perf_counter()
     for _ in range(steps):
-        ref.svdq_linear_from_x(*a)
+        fn(*a)
     dt = time.perf_counter() - t0
-    value = flops_per_step(rows, K, N) * steps / dt / 1e12
+    value = flops_per_step(rows, K, N, 0 if plain else R) * steps / dt / 1e12
     sample = f"each step: {rows} of {M} tokens of {args.workload} (all K, all N)"
     out = {
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": min(args.warmup, 1), "ms_per_step": round(1e3 * dt / steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "impl": "reference",
         "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "R": R},
+        "config": {"workload": args.workload, "M": M, "K": K, "N": N, "R": 0 if plain else R},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _blas_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -70,7 +70,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 5
+#define SVDQ_ABI_VERSION 6
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -112,16 +112,21 @@ int svdq_repack_weights(const uint8_t* wscales, int N, int K,
  * (svdq_quantize_plan); the K ranges' fp32 partial products of L are
  * summed in K-range order on chip, so results do not depend on timing.
  *   x           [M, ldx] bf16, first K columns used; ldx >= K, ldx % 8 == 0.
- *   smooth      [K] bf16 smoothing factor (multiplied, not divided).
- *   proj_down   [K, R] bf16.
- *   R           rank; only 128 is supported (else SVDQ_ERR_UNSUPPORTED).
+ *   smooth      [K] bf16 smoothing factor (multiplied, not divided), or
+ *               NULL: no smoothing (a factor of 1).
+ *   proj_down   [K, R] bf16 (NULL when R == 0).
+ *   R           rank: 128, or 0 for the plain NVFP4 layer without the
+ *               low-rank branch (Z-Image NVFP4 blog, the comfy-kitchen
+ *               deployment: weights quantized once, activations quantized
+ *               dynamically); then proj_down and lowrank are not used and
+ *               may be NULL.  Anything else gives SVDQ_ERR_UNSUPPORTED.
  *   qact        out, [M, K/2] bytes: E2M1 codes, low nibble = even k.
  *   ascales_tiled out, svdq_ascales_tiled_bytes(M, K) bytes: one e4m3
  *               scale per 16 k per row, scale = e4m3(amax/6), elements
  *               E2M1(v/scale); both rounded to nearest-even, saturating.
  *               Read its logical [M, K/16] form with svdq_unpack_scales.
  *   lowrank     out, [M, R] bf16: x @ proj_down accumulated in fp32 and
- *               rounded to bf16 (the raw x, not x * smooth).
+ *               rounded to bf16 (the raw x, not x * smooth); NULL if R == 0.
  * Limits: K % 64 == 0 (else SVDQ_ERR_UNSUPPORTED). */
 int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx,
                       const uint16_t* smooth, const uint16_t* proj_down, int R,
@@ -140,8 +145,11 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx,
  *   wscales_tiled  as written by svdq_repack_weights.
  *   wcscales [N], wtscale [1] (read on the device), proj_up [N, R],
  *   bias [N] or NULL: bf16.
+ *   R              128, or 0 without the low-rank branch (then lowrank and
+ *                  proj_up are not used and may be NULL; the term is 0).
  *   y              out, [M, ldy] bf16, ldy >= N, ldy % 8 == 0.
- * Limits: R == 128, K % 256 == 0, N % 32 == 0 (else SVDQ_ERR_UNSUPPORTED). */
+ * Limits: R in {0, 128}, K % 256 == 0, N % 32 == 0 (else
+ * SVDQ_ERR_UNSUPPORTED). */
 int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
                      const uint16_t* lowrank, const uint8_t* qweight,
                      const void* wscales_tiled, const uint16_t* wcscales,
@@ -152,7 +160,7 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
 /* ---- helpers ------------------------------------------------------------ */
 
 /* Launch shape svdq_quantize_act uses on the current device for an [M, K]
- * input: rows per tile (*bm, 64 or 128) and the number of K ranges per
+ * input with the low-rank branch (R = 128): rows per tile (*bm, 64 or 128) and the number of K ranges per
  * tile (*split: 1, 2, 4 or 8 CTAs of a cluster, at least 256 k each),
  * chosen to occupy the most SMs in one wave.  For inspection and tests;
  * needs a device. */

@@ -114,6 +114,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// LR: the layer has the low-rank branch (R = 128).  Without it (R = 0, the
+// plain NVFP4 layer) a tile has no low-rank slots, drain or MMAs and the
+// epilogue reads only the main accumulator.
+template <bool LR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/2] u8, box {128, 128}
                    const __grid_constant__ CUtensorMap tm_b,   // qweight [N, K/2] u8, box {128, 256}
@@ -155,8 +159,10 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_l);
-    prefetch_tmap(&tm_p);
+    if (LR) {
+      prefetch_tmap(&tm_l);
+      prefetch_tmap(&tm_p);
+    }
     prefetch_tmap(&tm_y);
     for (uint32_t s = 0; s < AB_SLOTS; ++s) {
       mbar_init(full_bar(s), 1);
@@ -197,7 +203,7 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
         const int mb = t % p.m_tiles;
         const int nb = t / p.m_tiles;
-        for (int st = 0; st < num_k + 2; ++st, ++it) {
+        for (int st = 0; st < num_k + (LR ? 2 : 0); ++st, ++it) {
           const uint32_t s = it % AB_SLOTS;
           const uint32_t ph = (it / AB_SLOTS) & 1u;
           if (!svdq_wait(empty_bar(s), ph ^ 1u, SITE_PROD)) {
@@ -258,6 +264,10 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
           tc_commit(sf_empty_bar(sf));
         }
         if (!ok) break;
+        if (!LR) {
+          tc_commit(tmem_full_bar);
+          continue;
+        }
         // The low-rank accumulator overlaps the scale-factor columns: let
         // every main MMA finish before the low-rank MMAs write there.
         tc_commit(drain_bar);
@@ -404,7 +414,12 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
         const int col = half * 128 + 16 * c;
         uint32_t acc[16], lr[16];
         tmem_ld_32x32b_x16(lane_base + TM_ACC + col, acc);
-        tmem_ld_32x32b_x16(lane_base + TM_LR + col, lr);
+        if (LR) {
+          tmem_ld_32x32b_x16(lane_base + TM_LR + col, lr);
+        } else {
+#pragma unroll
+          for (int z = 0; z < 16; ++z) lr[z] = 0u;   // +0.0f
+        }
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 8; ++i) {

@@ -46,6 +46,10 @@
 //               two independent groups side by side); it converts its 16
 //               smooth values once per stage; writes packed codes and tiled
 //               scales; afterwards reads L^T out of TMEM.
+// Without the low-rank branch (R = 0, the plain NVFP4 layer; template
+// parameter LR = false) the same kernel only quantizes: no proj_down, MMA,
+// TMEM or cluster, and a deeper ring of x stages.  A null smooth means no
+// smoothing (a factor of 1).
 // With split == 1 the tile's L is rounded to bf16 and written directly.
 // Otherwise every rank stages its fp32 partial in its own (idle) stage
 // ring, and after a cluster barrier each rank sums a 1/split slice of the
@@ -71,23 +75,29 @@ constexpr uint32_t SM_BYTES = STAGE_K * 2;         // 256 B
 constexpr int NUM_QWARPS = 16;
 constexpr int NUM_QTHREADS = NUM_QWARPS * 32;
 constexpr int NUM_THREADS = 64 + NUM_QTHREADS;
-constexpr uint32_t BAR_BYTES = 128;
+constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BUDGET = 227 * 1024;
 constexpr int PART_STRIDE = R + 4;     // floats per row of a staged partial (bank spread)
 constexpr int MAX_SPLIT = 8;
 
-template <int BM>
+// LR: the layer has the low-rank branch (R = 128); without it (R = 0, the
+// plain NVFP4 layer) a stage carries only x and smooth, there is no MMA,
+// no TMEM and no reduction, and the ring is deeper.
+template <int BM, bool LR = true>
 struct Shape {
   static constexpr uint32_t X_CHUNK = BM * 128;             // [BM rows x 64 k] bf16
   static constexpr uint32_t X_BYTES = 2 * X_CHUNK;
-  static constexpr uint32_t STAGE_BYTES = (X_BYTES + PD_BYTES + SM_BYTES + 1023u) & ~1023u;
+  static constexpr uint32_t PD_STAGE = LR ? PD_BYTES : 0u;
+  static constexpr uint32_t STAGE_BYTES = (X_BYTES + PD_STAGE + SM_BYTES + 1023u) & ~1023u;
   static constexpr int STAGES_FIT = static_cast<int>((SMEM_BUDGET - BAR_BYTES - 1024) / STAGE_BYTES);
-  static constexpr int STAGES = STAGES_FIT < 4 ? STAGES_FIT : 4;
+  static constexpr int MAX_STAGES = LR ? 4 : 8;
+  static constexpr int STAGES = STAGES_FIT < MAX_STAGES ? STAGES_FIT : MAX_STAGES;
   static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = BM;                 // 64 or 128 (powers of 2)
   static constexpr int ROWS_PER_THREAD = BM / 64;           // 1 or 2
   static_assert(STAGES >= 3, "at least three stages");
-  static_assert(BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partial fits the ring");
+  static_assert(!LR || BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partial fits the ring");
+  static_assert(16 * STAGES + 24 <= BAR_BYTES, "barriers fit");
 };
 
 constexpr uint32_t SITE_PROD = 0x20, SITE_MMA = 0x21, SITE_QUANT = 0x22, SITE_LFULL = 0x23;
@@ -181,12 +191,12 @@ __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
   return static_cast<uint64_t>(cvt_e2m1x8(qlo)) | (static_cast<uint64_t>(cvt_e2m1x8(qhi)) << 32);
 }
 
-template <int BM>
+template <int BM, bool LR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/64}, box {64, BM, 2}
                     const __grid_constant__ CUtensorMap tm_pd,   // proj_down {64, K, 2}, box {64, 128, 2}
                     const Params p) {
-  using S = Shape<BM>;
+  using S = Shape<BM, LR>;
   constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -197,7 +207,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
   // 128 B], smooth [128 k] bf16.
   auto s_x = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES; };
   auto s_pd = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES; };
-  auto s_sm = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES + PD_BYTES; };
+  auto s_sm = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES + S::PD_STAGE; };
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
   const uint32_t lfull_bar = s_bar + 16u * STAGES;
@@ -217,23 +227,23 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_x);
-    prefetch_tmap(&tm_pd);
+    if (LR) prefetch_tmap(&tm_pd);
     for (uint32_t s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1 + NUM_QWARPS);
+      mbar_init(empty_bar(s), (LR ? 1 : 0) + NUM_QWARPS);
     }
     mbar_init(lfull_bar, 1);
     mbar_init(final_bar, 1);
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (LR && warp == 1) {
     tmem_alloc(tmem_slot, S::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
+  const uint32_t tmem_base = LR ? *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr) : 0u;
   // Set-up above overlaps the previous kernel; global memory waits for it.
   griddep_wait();
   griddep_launch_dependents();
@@ -256,10 +266,11 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
         const int nc = c_end - kc0 < 2 ? 1 : 2;
         // Boxes are always delivered whole (zero fill past M and K); only
         // the smooth copy is cut to the chunks that exist.
-        mbar_arrive_expect_tx(full_bar(s), S::X_BYTES + PD_BYTES + nc * 128u);
+        const uint32_t sm_bytes = p.smooth != nullptr ? nc * 128u : 0u;
+        mbar_arrive_expect_tx(full_bar(s), S::X_BYTES + S::PD_STAGE + sm_bytes);
         tma_load_3d(s_x(s), &tm_x, 0, mb * BM, kc0, full_bar(s));
-        tma_load_3d(s_pd(s), &tm_pd, 0, kc0 * BKE, 0, full_bar(s));
-        bulk_load(s_sm(s), p.smooth + kc0 * BKE, nc * 128u, full_bar(s));
+        if (LR) tma_load_3d(s_pd(s), &tm_pd, 0, kc0 * BKE, 0, full_bar(s));
+        if (sm_bytes) bulk_load(s_sm(s), p.smooth + kc0 * BKE, sm_bytes, full_bar(s));
       }
       if (!ok) {
         const int n = i < STAGES ? i : STAGES;
@@ -270,7 +281,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (LR && lane == 0) {
       // ---------------------------------------------------- MMA issuer --
       // L^T[r, m] += sum_k proj_down[k, r] x[m, k]: A = proj_down stage
       // (MN-major: r contiguous; the two 64-r halves 16 KB apart, 8-row k
@@ -340,12 +351,16 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
       uint32_t sca = 0, scb = 0;
       if (active) {
         uint64_t nsm[8];
-        {
+        if (p.smooth != nullptr) {
           const uint4 sa = lds_v4(s_sm(s) + cg * 32);
           const uint4 sb = lds_v4(s_sm(s) + cg * 32 + 16);
           const uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
           for (int j = 0; j < 8; ++j) nsm[j] = bf16x2_to_pk(sw[j] ^ 0x80008000u);
+        } else {
+          // no smoothing: v = x, i.e. a factor of 1 (exact)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) nsm[j] = pk(-1.0f, -1.0f);
         }
         const uint32_t xs = s_x(s);
         const uint4 a0 = lds_v4(xs + xo0), a1 = lds_v4(xs + xo1);
@@ -390,7 +405,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
     }
-    l_ready = ok && __all_sync(0xFFFFFFFFu, svdq_wait(lfull_bar, 0, SITE_LFULL));
+    if (LR) l_ready = ok && __all_sync(0xFFFFFFFFu, svdq_wait(lfull_bar, 0, SITE_LFULL));
   }
 
   // ------------------------------------------------- low-rank readout --
@@ -403,7 +418,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
   constexpr int CW = BM / 4;     // 16 or 32 columns per warp
   const int mc = slice * CW;
   const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(lq * 32) << 16) + mc;
-  if (p.split == 1) {
+  if constexpr (!LR) {
+    // no low-rank branch: nothing to read out
+  } else if (p.split == 1) {
     if (is_q && l_ready) {
       tc_fence_after();
       uint32_t v[CW];
@@ -488,7 +505,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (LR && warp == 1) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, S::TMEM_COLS);

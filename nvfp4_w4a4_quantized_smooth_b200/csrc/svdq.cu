@@ -53,15 +53,25 @@ int device_setup(DeviceInfo** out) {
     for (auto& row : d.kq_clusters)
       for (int& v : row) v = -1;
     if (d.sm100) {
-      if (cudaFuncSetAttribute(svdq::kq::quantize_act_kernel<64>,
+      using namespace svdq;
+      if (cudaFuncSetAttribute(kq::quantize_act_kernel<64, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               svdq::kq::Shape<64>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(svdq::kq::quantize_act_kernel<128>,
+                               kq::Shape<64, true>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kq::quantize_act_kernel<128, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               svdq::kq::Shape<128>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(svdq::kg::w4a4_linear_kernel,
+                               kq::Shape<128, true>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kq::quantize_act_kernel<64, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               svdq::kg::SMEM_BYTES) != cudaSuccess)
+                               kq::Shape<64, false>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kq::quantize_act_kernel<128, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kq::Shape<128, false>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kg::w4a4_linear_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kg::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kg::w4a4_linear_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kg::SMEM_BYTES) != cudaSuccess)
         return SVDQ_ERR_CUDA;
     }
     if (g_encode == nullptr) {
@@ -145,8 +155,9 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const void* fn = bm == 128 ? reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<128>)
-                             : reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<64>);
+  const void* fn =
+      bm == 128 ? reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<128, true>)
+                : reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<64, true>);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -185,6 +196,31 @@ void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out) {
   *bm_out = best_bm;
   *split_out = best_split;
 }
+// Launch shape without the low-rank branch: no cluster and no reduction, so
+// the (BM, split) occupying the most SMs in one wave, ties to the tile
+// height that pads M least, then the taller tile and the smaller split.
+void kq_plan_plain(DeviceInfo* d, int M, int K, int* bm_out, int* split_out) {
+  const int chunks = K / svdq::kq::BKE;
+  int best_bm = 128, best_split = 1, best_ctas = -1, best_pad = 0;
+  for (int bm : {128, 64}) {
+    const int m_tiles = (M + bm - 1) / bm;
+    const int pad = m_tiles * bm - M;
+    for (int split = 1; split <= svdq::kq::MAX_SPLIT && (split == 1 || 4 * split <= chunks);
+         split *= 2) {
+      const int ctas = m_tiles * split;
+      if (ctas > d->num_sms) break;
+      if (ctas > best_ctas || (ctas == best_ctas && pad < best_pad)) {
+        best_ctas = ctas;
+        best_bm = bm;
+        best_split = split;
+        best_pad = pad;
+      }
+    }
+  }
+  *bm_out = best_bm;
+  *split_out = best_split;
+}
+
 // One thread waits, through the same bounded wait the layer's kernels use,
 // on an mbarrier that completes only if `arrive` is set.  With arrive = 0
 // nothing completes it, so the wait runs out after the current limit and
@@ -261,28 +297,36 @@ int svdq_repack_weights(const uint8_t* wscales, int N, int K, void* wscales_tile
 int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* smooth,
                       const uint16_t* proj_down, int R, uint8_t* qact, void* ascales_tiled,
                       uint16_t* lowrank, void* stream) {
-  if (!x || !smooth || !proj_down || !qact || !ascales_tiled || !lowrank)
+  const bool lr = R != 0;
+  if (!x || !qact || !ascales_tiled || (lr && (!proj_down || !lowrank)))
     return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || K < 16 || K % 16 || ldx < K) return SVDQ_ERR_SHAPE;
-  if (R != svdq::kq::R || K % 64) return SVDQ_ERR_UNSUPPORTED;
-  if (!aligned(x, 16) || !aligned(smooth, 16) || !aligned(proj_down, 16) || !aligned(qact, 16) ||
-      !aligned(ascales_tiled, 16) || !aligned(lowrank, 16) || ldx % 8)
+  if ((R != svdq::kq::R && R != 0) || K % 64) return SVDQ_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || (smooth && !aligned(smooth, 16)) || !aligned(qact, 16) ||
+      !aligned(ascales_tiled, 16) || (lr && (!aligned(proj_down, 16) || !aligned(lowrank, 16))) ||
+      ldx % 8)
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
   if (int st = device_setup(&d)) return st;
 
   const int chunks = K / svdq::kq::BKE;
   int bm = 0, split = 0;
-  kq_plan(d, M, K, &bm, &split);
+  if (lr)
+    kq_plan(d, M, K, &bm, &split);
+  else
+    kq_plan_plain(d, M, K, &bm, &split);
   const int m_tiles = (M + bm - 1) / bm;
 
   // x viewed as {64 k, M rows, K/64 chunks} and proj_down as {64 r, K,
   // 2 halves of R}, so that one box carries a whole 128-k stage.
   CUtensorMap tm_x, tm_pd;
   if (make_tmap3(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, svdq::kq::BKE, M, chunks,
-                 static_cast<uint64_t>(ldx) * 2, svdq::kq::BKE * 2, svdq::kq::BKE, bm, 2) ||
-      make_tmap3(&tm_pd, proj_down, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, K, 2,
-                 static_cast<uint64_t>(R) * 2, 128, 64, svdq::kq::STAGE_K, 2))
+                 static_cast<uint64_t>(ldx) * 2, svdq::kq::BKE * 2, svdq::kq::BKE, bm, 2))
+    return SVDQ_ERR_CUDA;
+  if (!lr)
+    tm_pd = tm_x;   // not read
+  else if (make_tmap3(&tm_pd, proj_down, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, K, 2,
+                      static_cast<uint64_t>(R) * 2, 128, 64, svdq::kq::STAGE_K, 2))
     return SVDQ_ERR_CUDA;
 
   svdq::kq::Params p;
@@ -299,21 +343,29 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(split, m_tiles, 1);
   cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes =
-      bm == 128 ? svdq::kq::Shape<128>::SMEM_BYTES : svdq::kq::Shape<64>::SMEM_BYTES;
+  using svdq::kq::Shape;
+  using svdq::kq::quantize_act_kernel;
+  cfg.dynamicSmemBytes = lr ? (bm == 128 ? Shape<128, true>::SMEM_BYTES : Shape<64, true>::SMEM_BYTES)
+                            : (bm == 128 ? Shape<128, false>::SMEM_BYTES : Shape<64, false>::SMEM_BYTES);
   cfg.stream = static_cast<cudaStream_t>(stream);
+  // The K ranges of a tile form a cluster only when their L partials are
+  // summed (low-rank branch).
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = split;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = split;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  const cudaError_t e =
-      bm == 128 ? cudaLaunchKernelEx(&cfg, svdq::kq::quantize_act_kernel<128>, tm_x, tm_pd, p)
-                : cudaLaunchKernelEx(&cfg, svdq::kq::quantize_act_kernel<64>, tm_x, tm_pd, p);
+  cfg.numAttrs = lr ? 2 : 1;
+  cudaError_t e;
+  if (lr)
+    e = bm == 128 ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<128, true>, tm_x, tm_pd, p)
+                  : cudaLaunchKernelEx(&cfg, quantize_act_kernel<64, true>, tm_x, tm_pd, p);
+  else
+    e = bm == 128 ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<128, false>, tm_x, tm_pd, p)
+                  : cudaLaunchKernelEx(&cfg, quantize_act_kernel<64, false>, tm_x, tm_pd, p);
   if (e != cudaSuccess) return SVDQ_ERR_CUDA;
   return launch_status();
 }
@@ -322,14 +374,15 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
                      const uint8_t* qweight, const void* wscales_tiled, const uint16_t* wcscales,
                      const uint16_t* wtscale, const uint16_t* proj_up, const uint16_t* bias, int M,
                      int N, int K, int R, uint16_t* y, int ldy, void* stream) {
-  if (!qact || !ascales_tiled || !lowrank || !qweight || !wscales_tiled || !wcscales || !wtscale ||
-      !proj_up || !y)
+  const bool lr = R != 0;
+  if (!qact || !ascales_tiled || !qweight || !wscales_tiled || !wcscales || !wtscale || !y ||
+      (lr && (!lowrank || !proj_up)))
     return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 16 || K % 16 || ldy < N) return SVDQ_ERR_SHAPE;
-  if (R != 128 || K % svdq::kg::BK || N % 32) return SVDQ_ERR_UNSUPPORTED;
-  if (!aligned(qact, 16) || !aligned(ascales_tiled, 16) || !aligned(lowrank, 16) ||
-      !aligned(qweight, 16) || !aligned(wscales_tiled, 16) || !aligned(wcscales, 16) ||
-      !aligned(wtscale, 2) || !aligned(proj_up, 16) || (bias && !aligned(bias, 16)) ||
+  if ((R != 128 && R != 0) || K % svdq::kg::BK || N % 32) return SVDQ_ERR_UNSUPPORTED;
+  if (!aligned(qact, 16) || !aligned(ascales_tiled, 16) || !aligned(qweight, 16) ||
+      !aligned(wscales_tiled, 16) || !aligned(wcscales, 16) || !aligned(wtscale, 2) ||
+      (lr && (!aligned(lowrank, 16) || !aligned(proj_up, 16))) || (bias && !aligned(bias, 16)) ||
       !aligned(y, 16) || ldy % 8)
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
@@ -341,13 +394,18 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
                 svdq::kg::BM) ||
       make_tmap(&tm_b, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, N, kb, svdq::kg::BK_BYTES,
                 svdq::kg::BN) ||
-      make_tmap(&tm_l, lowrank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, M,
-                static_cast<uint64_t>(R) * 2, 64, svdq::kg::BM) ||
-      make_tmap(&tm_p, proj_up, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, N,
-                static_cast<uint64_t>(R) * 2, 64, svdq::kg::BN) ||
       make_tmap(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(ldy) * 2,
                 svdq::kg::OUT_COLS, 32))
     return SVDQ_ERR_CUDA;
+  if (!lr) {
+    tm_l = tm_a;   // not read
+    tm_p = tm_b;
+  } else if (make_tmap(&tm_l, lowrank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, M,
+                       static_cast<uint64_t>(R) * 2, 64, svdq::kg::BM) ||
+             make_tmap(&tm_p, proj_up, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, N,
+                       static_cast<uint64_t>(R) * 2, 64, svdq::kg::BN)) {
+    return SVDQ_ERR_CUDA;
+  }
 
   svdq::kg::Params p;
   p.ascales_tiled = static_cast<const uint8_t*>(ascales_tiled);
@@ -373,9 +431,12 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, svdq::kg::w4a4_linear_kernel, tm_a, tm_b, tm_l, tm_p, tm_y, p) !=
-      cudaSuccess)
-    return SVDQ_ERR_CUDA;
+  const cudaError_t e =
+      lr ? cudaLaunchKernelEx(&cfg, svdq::kg::w4a4_linear_kernel<true>, tm_a, tm_b, tm_l, tm_p,
+                              tm_y, p)
+         : cudaLaunchKernelEx(&cfg, svdq::kg::w4a4_linear_kernel<false>, tm_a, tm_b, tm_l, tm_p,
+                              tm_y, p);
+  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
   return launch_status();
 }
 

@@ -29,7 +29,7 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 5
+ABI_VERSION = 6
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
 
@@ -135,46 +135,60 @@ def repack_weights(wscales: torch.Tensor, out: Optional[torch.Tensor] = None,
     return out
 
 
-def quantize_act(x: torch.Tensor, smooth: torch.Tensor, proj_down: torch.Tensor,
+def quantize_act(x: torch.Tensor, smooth: Optional[torch.Tensor],
+                 proj_down: Optional[torch.Tensor],
                  qact: Optional[torch.Tensor] = None,
                  ascales_tiled: Optional[torch.Tensor] = None,
                  lowrank: Optional[torch.Tensor] = None, stream=None):
-    """x [M, K] bf16 (row stride may exceed K) -> (qact, ascales_tiled, lowrank)."""
+    """x [M, K] bf16 (row stride may exceed K) -> (qact, ascales_tiled, lowrank).
+
+    smooth None: no smoothing.  proj_down None: the plain NVFP4 layer
+    (R = 0); lowrank is then None."""
     _need(x, torch.bfloat16, "x", 2)
-    _need(smooth, torch.bfloat16, "smooth", 1)
-    _need(proj_down, torch.bfloat16, "proj_down", 2)
+    if smooth is not None:
+        _need(smooth, torch.bfloat16, "smooth", 1)
+        smooth = smooth.contiguous()
+    if proj_down is not None:
+        _need(proj_down, torch.bfloat16, "proj_down", 2)
+        proj_down = proj_down.contiguous()
     if x.stride(1) != 1:
         raise ValueError("x must have unit stride along K")
     M, K = x.shape
-    R = proj_down.shape[1]
+    R = 0 if proj_down is None else proj_down.shape[1]
     dev = x.device
     if qact is None:
         qact = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
     if ascales_tiled is None:
         ascales_tiled = torch.empty(max(ascales_tiled_bytes(M, K), 1), dtype=torch.uint8,
                                     device=dev)
-    if lowrank is None:
+    if lowrank is None and R:
         lowrank = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
-    _check(_lib.svdq_quantize_act(_ptr(x), M, K, x.stride(0), _ptr(smooth.contiguous()),
-                                  _ptr(proj_down.contiguous()), R, _ptr(qact),
-                                  _ptr(ascales_tiled), _ptr(lowrank), _stream(stream)),
+    _check(_lib.svdq_quantize_act(_ptr(x), M, K, x.stride(0), _ptr(smooth), _ptr(proj_down), R,
+                                  _ptr(qact), _ptr(ascales_tiled), _ptr(lowrank if R else None),
+                                  _stream(stream)),
            "svdq_quantize_act")
-    return qact, ascales_tiled, lowrank
+    return qact, ascales_tiled, (lowrank if R else None)
 
 
-def w4a4_linear(qact: torch.Tensor, ascales_tiled: torch.Tensor, lowrank: torch.Tensor,
-                qweight: torch.Tensor, wscales_tiled: torch.Tensor, wcscales: torch.Tensor,
-                wtscale: torch.Tensor, proj_up: torch.Tensor, bias: Optional[torch.Tensor],
+def w4a4_linear(qact: torch.Tensor, ascales_tiled: torch.Tensor,
+                lowrank: Optional[torch.Tensor], qweight: torch.Tensor,
+                wscales_tiled: torch.Tensor, wcscales: torch.Tensor, wtscale: torch.Tensor,
+                proj_up: Optional[torch.Tensor], bias: Optional[torch.Tensor],
                 y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """The block-scaled FP4 GEMM with the fused epilogue -> y [M, N] bf16."""
+    """The block-scaled FP4 GEMM with the fused epilogue -> y [M, N] bf16.
+
+    lowrank and proj_up None: the plain NVFP4 layer (R = 0)."""
     _need(qact, torch.uint8, "qact", 2)
     _need(qweight, torch.uint8, "qweight", 2)
-    _need(lowrank, torch.bfloat16, "lowrank", 2)
-    _need(proj_up, torch.bfloat16, "proj_up", 2)
+    if (lowrank is None) != (proj_up is None):
+        raise ValueError("lowrank and proj_up go together (both None for R = 0)")
+    if lowrank is not None:
+        _need(lowrank, torch.bfloat16, "lowrank", 2)
+        _need(proj_up, torch.bfloat16, "proj_up", 2)
     M = qact.shape[0]
     K = qact.shape[1] * 2
     N = qweight.shape[0]
-    R = proj_up.shape[1]
+    R = 0 if proj_up is None else proj_up.shape[1]
     if y is None:
         y = torch.empty(M, N, dtype=torch.bfloat16, device=qact.device)
     _check(_lib.svdq_w4a4_linear(_ptr(qact), _ptr(ascales_tiled), _ptr(lowrank),

@@ -113,6 +113,10 @@ WORKLOADS = {
     "ffn_w3_m4352_k3840_n10240": (TOKENS, HIDDEN, FFN),
     "ffn_w2_m4352_k10240_n3840": (TOKENS, FFN, HIDDEN),
 }
+# The plain NVFP4 layer (no low-rank branch, no smoothing) at the qkv shape.
+PLAIN_PREFIX = "nvfp4_"
+WORKLOADS[PLAIN_PREFIX + "qkv_m4352_k3840_n11520"] = (TOKENS, HIDDEN, 3 * HIDDEN)
+
 OUT_PROJ_SWEEP_M = (16, 64, 256, 1024, 4352, 17408)
 for _m in OUT_PROJ_SWEEP_M:
     WORKLOADS[f"out_m{_m}_k3840_n3840"] = (_m, HIDDEN, HIDDEN)
@@ -172,6 +176,8 @@ def workload_seed(name: str, layer: int = 0) -> int:
         base = 3000 + OUT_PROJ_SWEEP_M.index(int(name.split("_")[1][1:]))
     if base is None and name.startswith("dit_"):
         base = 4000
+    if base is None and name.startswith(PLAIN_PREFIX):
+        base = 5000
     if base is None:
         raise KeyError(name)
     return base + 100 * layer

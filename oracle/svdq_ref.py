@@ -129,3 +129,28 @@ def svdq_linear_from_x(x_bits, smooth_bits, proj_down_bits, qweight, wscales,
     y = w4a4_linear(qact, ascales, qweight, wscales, wcscales_bits,
                     wtscale_bits, proj_up_bits, bias_bits, L)
     return y, qact, ascales, L
+
+
+BF16_ONE = 0x3F80
+
+
+def plain_linear_from_x(x_bits, qweight, wscales, wcscales_bits, wtscale_bits, bias_bits,
+                        smooth_bits=None):
+    """The layer without the low-rank branch (R = 0): the plain NVFP4 linear
+    of the Z-Image NVFP4 blog's comfy-kitchen deployment (weights quantized
+    once, activations quantized dynamically at inference).
+
+        y = scaled_mma(quant(x * smooth), qweight, ascales, wscales)
+            * wtscale * wcscales + bias
+
+    with smooth = 1 (no smoothing) when ``smooth_bits`` is None.  Returns
+    (y float64 [M, N], qact, ascales).
+    """
+    M, K = x_bits.shape
+    N = qweight.shape[0]
+    if smooth_bits is None:
+        smooth_bits = np.full(K, BF16_ONE, dtype=np.uint16)
+    qact, ascales = quantize_act(x_bits, smooth_bits)
+    y = w4a4_linear(qact, ascales, qweight, wscales, wcscales_bits, wtscale_bits,
+                    np.zeros((N, 0), dtype=np.uint16), bias_bits, np.zeros((M, 0)))
+    return y, qact, ascales

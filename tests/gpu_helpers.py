@@ -84,6 +84,32 @@ def oracle_y(L: synth.LayerOperands, rows=None, cols=None, x=None):
     return y, qact, asc, Lr
 
 
+def gpu_plain_layer(L: synth.LayerOperands, with_smooth: bool):
+    """The layer without the low-rank branch (R = 0) on the GPU."""
+    s = svdq()
+    d = to_dev(L)
+    M, K = d["x"].shape
+    wt = s.repack_weights(d["wscales"])
+    qact, asc, lr = s.quantize_act(d["x"], d["smooth"] if with_smooth else None, None)
+    assert lr is None
+    y = s.w4a4_linear(qact, asc, None, d["qweight"], wt, d["wcscales"], d["wtscale"], None,
+                      d["bias"])
+    s.check_device_error()
+    asc_logical = s.unpack_scales(asc, M, K)
+    torch.cuda.synchronize()
+    return dict(qact=qact.cpu(), ascales=asc_logical.cpu(), y=y.cpu())
+
+
+def oracle_plain_y(L: synth.LayerOperands, with_smooth: bool, rows=None):
+    xb = bits(L.x)
+    if rows is not None:
+        xb = xb[rows]
+    bb = None if L.bias is None else bits(L.bias)
+    return ref.plain_linear_from_x(xb, bits(L.qweight), bits(L.wscales), bits(L.wcscales),
+                                   bits(L.wtscale), bb,
+                                   smooth_bits=bits(L.smooth) if with_smooth else None)
+
+
 def assert_y_close(y_gpu_bf16: torch.Tensor, y_ref: np.ndarray, what=""):
     yg = y_gpu_bf16.to(torch.float64).numpy()
     assert yg.shape == y_ref.shape

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(svdq):
 
 
 def test_abi_version_and_status_strings(svdq):
-    assert svdq.abi_version() == 5 == svdq.ABI_VERSION
+    assert svdq.abi_version() == 6 == svdq.ABI_VERSION
     for st in range(8):
         s = svdq._lib.svdq_status_string(st).decode()
         assert s.startswith("SVDQ")
@@ -100,6 +100,18 @@ def test_argument_checks_fail_before_any_device_work(svdq):
                                  None) == svdq.SVDQ_ERR_ALIGNMENT
     assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, odd, 16, 64,
                                 256, 128, fake, 64, None) == svdq.SVDQ_ERR_ALIGNMENT
+    # R = 0 (no low-rank branch): proj_down, lowrank, proj_up and smooth may
+    # be null; the other checks still apply
+    assert lib.svdq_quantize_act(fake, 0, 64, 64, None, None, 0, fake, fake, None,
+                                 None) == svdq.SVDQ_ERR_SHAPE
+    assert lib.svdq_quantize_act(fake, 16, 64, 64, None, None, 0, None, fake, None,
+                                 None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_quantize_act(fake, 16, 64, 64, None, None, 128, fake, fake, fake,
+                                 None) == svdq.SVDQ_ERR_INVALID_ARG      # R = 128 needs proj_down
+    assert lib.svdq_w4a4_linear(fake, fake, None, fake, fake, fake, fake, None, None, 16, 48,
+                                256, 0, fake, 48, None) == svdq.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_w4a4_linear(fake, fake, None, fake, fake, fake, fake, None, None, 16, 64,
+                                256, 128, fake, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
     # scale unpack: only the two documented tile orders
     for kind in (-1, 2):
         assert lib.svdq_unpack_scales(fake, 16, 64, kind, fake, None) == svdq.SVDQ_ERR_INVALID_ARG

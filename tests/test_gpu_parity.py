@@ -205,6 +205,28 @@ def test_linear_parity(M, K, N):
     H.assert_y_close(r["y"], y_ref, f"M={M} K={K} N={N}")
 
 
+@pytest.mark.parametrize("M,K,N,with_smooth", [(300, 512, 384, False), (128, 1024, 512, True),
+                                               (16, 3840, 3840, False), (1000, 768, 1280, True)])
+def test_plain_nvfp4_layer(M, K, N, with_smooth):
+    # R = 0: no low-rank branch; without smooth, x is quantized as it is.
+    L = synth.make_layer(M, K, N, seed=3 * M + K + 7 * N + with_smooth)
+    r = H.gpu_plain_layer(L, with_smooth)
+    y_ref, q_ref, a_ref = H.oracle_plain_y(L, with_smooth)
+    H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, "plain quant")
+    H.assert_y_close(r["y"], y_ref, f"plain M={M} K={K} N={N}")
+
+
+def test_plain_nvfp4_layer_full_size_qkv():
+    name = "qkv_m4352_k3840_n11520"
+    M, K, N = synth.WORKLOADS[name]
+    L = synth.make_layer(M, K, N, seed=synth.workload_seed(name))
+    r = H.gpu_plain_layer(L, False)
+    rows = H.sample_rows(M, 32, seed=5)
+    y_ref, q_ref, a_ref = H.oracle_plain_y(L, False, rows=rows)
+    H.assert_quant_exact(r["qact"][rows], r["ascales"][rows], q_ref, a_ref, "plain qkv quant")
+    H.assert_y_close(r["y"][rows], y_ref, "plain qkv")
+
+
 def test_linear_without_bias():
     L = synth.make_layer(64, 512, 256, seed=21, with_bias=False)
     r = H.gpu_layer(L)

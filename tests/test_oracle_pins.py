@@ -432,6 +432,54 @@ def test_integer_grid_invariant():
     assert np.all(np.mod(y * 4, 1) == 0)        # multiples of 0.25
 
 
+def test_plain_layer_integer_grid_exact():
+    # The layer without the low-rank branch and without smoothing: every x
+    # group on the E2M1 grid with amax 6 and unit weight scales give an exact
+    # rational matmul of the codes, scaled by wtscale * wcscales, plus bias.
+    rng = np.random.default_rng(11)
+    M, K, N = 4, 96, 6
+    codes_x = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    codes_x[:, ::16] = 15                                 # amax 6 (as -6) in every group
+    x = nv.decode_e2m1(codes_x)
+    xb = bf16_bits_of(x.ravel()).reshape(M, K)
+    qw = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    ws = np.full((K // 16, N), 0x38, dtype=np.uint8)      # 1.0
+    wc = bf16_bits_of([0.5, 1.0, 2.0, 0.25, 4.0, 1.5])
+    wt = bf16_bits_of([0.125])
+    bias = bf16_bits_of([1.0, -2.0, 0.5, 0.0, 3.0, -0.25])
+    y, qact, asc = ref.plain_linear_from_x(xb, qw, ws, wc, wt, bias)
+    assert np.all(asc == 0x38)
+    assert np.array_equal(nv.unpack_nibbles(qact), codes_x)
+    w = nv.decode_e2m1(nv.unpack_nibbles(qw))
+    cs = [0.5, 1.0, 2.0, 0.25, 4.0, 1.5]
+    bs = [1.0, -2.0, 0.5, 0.0, 3.0, -0.25]
+    exact = np.array([[sum(Fraction(float(x[m, k])) * Fraction(float(w[n, k])) for k in range(K))
+                       * Fraction(1, 8) * Fraction(cs[n]) + Fraction(bs[n])
+                       for n in range(N)] for m in range(M)])
+    assert np.array_equal(y, exact.astype(np.float64))
+
+
+def test_plain_layer_is_the_layer_with_unit_smooth_and_no_lowrank():
+    # No smooth = a factor of 1 (x * 1 is exact); R = 0 = a zero low-rank term.
+    L = synth.make_layer(6, 64, 10, R=4, seed=12)
+    b = synth.bits
+    K, N = 64, 10
+    y0, q0, a0 = ref.plain_linear_from_x(b(L.x), b(L.qweight), b(L.wscales), b(L.wcscales),
+                                         b(L.wtscale), b(L.bias))
+    # the smoothed layer's quantizer on x * 1, and a zero low-rank product
+    y1, q1, a1, _ = ref.svdq_linear_from_x(
+        b(L.x), bf16_bits_of([1.0] * K), bf16_bits_of([0.0] * K * 4).reshape(K, 4),
+        b(L.qweight), b(L.wscales), b(L.wcscales), b(L.wtscale),
+        bf16_bits_of([0.0] * N * 4).reshape(N, 4), b(L.bias))
+    assert np.array_equal(q0, q1) and np.array_equal(a0, a1)
+    assert np.array_equal(y0, y1)
+    # with a smooth factor given, the codes are those of x * smooth
+    y2, q2, a2 = ref.plain_linear_from_x(b(L.x), b(L.qweight), b(L.wscales), b(L.wcscales),
+                                         b(L.wtscale), b(L.bias), smooth_bits=b(L.smooth))
+    q3, a3 = ref.quantize_act(b(L.x), b(L.smooth))
+    assert np.array_equal(q2, q3) and np.array_equal(a2, a3)
+
+
 def test_lowrank_uses_raw_x():
     # The low-rank branch is (x @ proj_down), not (x * smooth) @ proj_down.
     L = synth.make_layer(4, 32, 8, R=4, seed=9)
