@@ -55,6 +55,9 @@ def parse_args(argv=None):
                     help="skip the end-to-end (host buffer) measurement")
     ap.add_argument("--no-graph", action="store_true",
                     help="stack workloads: skip the CUDA-graph replay measurement")
+    ap.add_argument("--unfused-w2", action="store_true",
+                    help="stack workloads: form w2's input with svdq_silu_mul in HBM, then "
+                         "quantize it (for comparison with the fused activation kernel)")
     return ap.parse_args(argv)
 
 
@@ -466,10 +469,10 @@ def stack_flops(M=None):
 
 def bench_stack(args, world, rank, local):
     """One step = all 150 linears of the 30-block stack (qkv, out, w1, w3,
-    w2 per block; quantize + GEMM each) back to back in one stream, at
-    M = 4352 tokens.  Block inputs and the w2 inputs (silu(y_w1) * y_w3 of
-    the same block, formed once before timing) are resident; weights
-    (3.2 GB) stream from HBM, so no L2 flush is needed."""
+    w2 per block; quantize + GEMM each) back to back in one stream.  Block
+    inputs are resident; w2's input silu(y_w1) * y_w3 is formed inside the
+    step by the fused activation kernel from that block's w1 / w3 outputs;
+    weights (3.2 GB) stream from HBM, so no L2 flush is needed."""
     import torch
     from nvfp4_w4a4_quantized_smooth_b200 import build as b
     if rank == 0:
@@ -508,19 +511,33 @@ def bench_stack(args, world, rank, local):
             svdq.w4a4_linear(qa, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
                              w.proj_up, w.bias, y=y, stream=stream)
 
-        for blk in blocks:   # the w2 inputs, from the GPU's own outputs
-            linear(blk["x"], blk["w"]["w1"], ybuf["w1"])
-            linear(blk["x"], blk["w"]["w3"], ybuf["w3"])
-            blk["h"] = svdq.silu_mul(ybuf["w1"], ybuf["w3"], stream=stream)
+        hbuf = torch.empty_like(ybuf["w1"]) if args.unfused_w2 else None
+
+        def w2_linear(w, y):
+            # w2's input silu(y_w1) * y_w3 is formed on chip by the
+            # activation kernel (never written to HBM), or, for comparison,
+            # in HBM by svdq_silu_mul and then quantized
+            qa, asc, lr = act[w.K]
+            if hbuf is not None:
+                svdq.silu_mul(ybuf["w1"], ybuf["w3"], out=hbuf, stream=stream)
+                svdq.quantize_act(hbuf, w.smooth, w.proj_down, qact=qa, ascales_tiled=asc,
+                                  lowrank=lr, stream=stream)
+            else:
+                svdq.silu_mul_quantize_act(ybuf["w1"], ybuf["w3"], w.smooth, w.proj_down,
+                                           qact=qa, ascales_tiled=asc, lowrank=lr, stream=stream)
+            svdq.w4a4_linear(qa, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
+                             w.proj_up, w.bias, y=y, stream=stream)
 
         def step(evs=None):
             j = 0
             for blk in blocks:
                 for n in order:
-                    x = blk["h"] if n == "w2" else blk["x"]
                     if evs is not None:
                         evs[j].record(stream)
-                    linear(x, blk["w"][n], ybuf[n])
+                    if n == "w2":
+                        w2_linear(blk["w"][n], ybuf[n])
+                    else:
+                        linear(blk["x"], blk["w"][n], ybuf[n])
                     j += 1
             if evs is not None:
                 evs[j].record(stream)
@@ -598,6 +615,8 @@ def bench_stack(args, world, rank, local):
         "data": "synthetic (seeded; random weights of the stack's shapes)",
         "config": {"workload": args.workload, "M": M, "blocks": len(blocks),
                    "linears_per_step": n_lin, "R": R, "cuda_graph": graph,
+                   "w2_input": "svdq_silu_mul then svdq_quantize_act" if args.unfused_w2
+                               else "formed on chip (svdq_silu_mul_quantize_act)",
                    "parallelism": f"dp{world} (independent token batches per GPU)",
                    "l2": "weights of 150 linears (3.2 GB) stream from HBM every step",
                    "per_linear": per_linear},
@@ -608,7 +627,7 @@ def bench_stack(args, world, rank, local):
                      "peak_source": f"{peak_src} bf16 sustained x {FP4_OVER_BF16:g} (nominal "
                                     "FP4:BF16 dense ratio; a step of ~16 ms is a sustained load)"},
         "e2e": None,
-        "gpu_launches": 2 * n_lin * steps,
+        "gpu_launches": (2 * n_lin + (len(blocks) if args.unfused_w2 else 0)) * steps,
         "clocks": clocks.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

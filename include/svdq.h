@@ -70,7 +70,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 6
+#define SVDQ_ABI_VERSION 7
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -132,6 +132,23 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx,
                       const uint16_t* smooth, const uint16_t* proj_down, int R,
                       uint8_t* qact, void* ascales_tiled, uint16_t* lowrank,
                       void* stream);
+
+/* Activation side of the w2 linear of a DiT feed-forward block, whose input
+ * is silu(w1 x) * (w3 x): reads a = w1's output and b = w3's output, forms
+ * x = silu(a) * b on chip with the same fp32 arithmetic and bf16 rounding
+ * as svdq_silu_mul, and writes quant(x * smooth) and x @ proj_down exactly
+ * as svdq_quantize_act does for that x (x itself is never written to
+ * global memory).  This is the step just before w2 on the feed-forward
+ * path of the DiT whose linears the layer replaces (w2(silu(w1 x) * w3 x),
+ * as svdq_silu_mul forms it); it saves writing and re-reading x.
+ *   a, b        [M, ld] bf16 with the same row stride, first K columns used;
+ *               ld >= K, ld % 8 == 0.
+ *   the other arguments and the statuses as svdq_quantize_act (R = 128 or
+ *   0; smooth may be NULL). */
+int svdq_silu_mul_quantize_act(const uint16_t* a, const uint16_t* b, int M, int K, int ld,
+                               const uint16_t* smooth, const uint16_t* proj_down, int R,
+                               uint8_t* qact, void* ascales_tiled, uint16_t* lowrank,
+                               void* stream);
 
 /* Block-scaled FP4 GEMM with the fused epilogue (model card runtime
  * formula):

@@ -50,6 +50,11 @@
 // parameter LR = false) the same kernel only quantizes: no proj_down, MMA,
 // TMEM or cluster, and a deeper ring of x stages.  A null smooth means no
 // smoothing (a factor of 1).
+// With SILU the input is x = silu(a) * b (bf16) of two [M, K] tensors, the
+// w2 input of a DiT feed-forward block: each stage also brings the b tile,
+// the quantizer threads form x in place of a (the same function and
+// rounding as svdq_silu_mul), and the MMA waits for every quantizer warp's
+// part before reading it; x itself is never written to global memory.
 // With split == 1 the tile's L is rounded to bf16 and written directly.
 // Otherwise every rank stages its fp32 partial in its own (idle) stage
 // ring, and after a cluster barrier each rank sums a 1/split slice of the
@@ -83,12 +88,17 @@ constexpr int MAX_SPLIT = 8;
 // LR: the layer has the low-rank branch (R = 128); without it (R = 0, the
 // plain NVFP4 layer) a stage carries only x and smooth, there is no MMA,
 // no TMEM and no reduction, and the ring is deeper.
-template <int BM, bool LR = true>
+// SILU: the input is silu(a) * b of two [M, K] tensors (w2's input in a
+// DiT feed-forward block), formed in shared memory; a stage then also holds
+// the b tile.
+template <int BM, bool LR = true, bool SILU = false>
 struct Shape {
   static constexpr uint32_t X_CHUNK = BM * 128;             // [BM rows x 64 k] bf16
   static constexpr uint32_t X_BYTES = 2 * X_CHUNK;
+  static constexpr uint32_t Y_STAGE = SILU ? X_BYTES : 0u;  // the b tile
   static constexpr uint32_t PD_STAGE = LR ? PD_BYTES : 0u;
-  static constexpr uint32_t STAGE_BYTES = (X_BYTES + PD_STAGE + SM_BYTES + 1023u) & ~1023u;
+  static constexpr uint32_t STAGE_BYTES =
+      (X_BYTES + Y_STAGE + PD_STAGE + SM_BYTES + 1023u) & ~1023u;
   static constexpr int STAGES_FIT = static_cast<int>((SMEM_BUDGET - BAR_BYTES - 1024) / STAGE_BYTES);
   static constexpr int MAX_STAGES = LR ? 4 : 8;
   static constexpr int STAGES = STAGES_FIT < MAX_STAGES ? STAGES_FIT : MAX_STAGES;
@@ -97,7 +107,7 @@ struct Shape {
   static constexpr int ROWS_PER_THREAD = BM / 64;           // 1 or 2
   static_assert(STAGES >= 3, "at least three stages");
   static_assert(!LR || BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partial fits the ring");
-  static_assert(16 * STAGES + 24 <= BAR_BYTES, "barriers fit");
+  static_assert(24 * STAGES + 24 <= BAR_BYTES, "barriers fit");
 };
 
 constexpr uint32_t SITE_PROD = 0x20, SITE_MMA = 0x21, SITE_QUANT = 0x22, SITE_LFULL = 0x23;
@@ -191,12 +201,13 @@ __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
   return static_cast<uint64_t>(cvt_e2m1x8(qlo)) | (static_cast<uint64_t>(cvt_e2m1x8(qhi)) << 32);
 }
 
-template <int BM, bool LR>
+template <int BM, bool LR, bool SILU>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/64}, box {64, BM, 2}
+quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64, M, K/64}, box {64, BM, 2}
+                    const __grid_constant__ CUtensorMap tm_y,    // b {64, M, K/64} (SILU only)
                     const __grid_constant__ CUtensorMap tm_pd,   // proj_down {64, K, 2}, box {64, 128, 2}
                     const Params p) {
-  using S = Shape<BM, LR>;
+  using S = Shape<BM, LR, SILU>;
   constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -206,11 +217,17 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
   // Stage layout: x [chunk][BM rows x 128 B], proj_down [r half][128 k x
   // 128 B], smooth [128 k] bf16.
   auto s_x = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES; };
-  auto s_pd = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES; };
-  auto s_sm = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES + S::PD_STAGE; };
+  auto s_y = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES; };
+  auto s_pd = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES + S::Y_STAGE; };
+  auto s_sm = [&](uint32_t s) {
+    return s_ring + s * S::STAGE_BYTES + S::X_BYTES + S::Y_STAGE + S::PD_STAGE;
+  };
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
-  const uint32_t lfull_bar = s_bar + 16u * STAGES;
+  // SILU: the x slot holds silu(a) * b once every quantizer warp has written
+  // its part (the MMA reads it then).
+  auto h_ready_bar = [&](uint32_t s) { return s_bar + 8u * (2 * STAGES + s); };
+  const uint32_t lfull_bar = s_bar + 8u * (3 * STAGES);
   const uint32_t final_bar = lfull_bar + 8u;
   const uint32_t tmem_slot = lfull_bar + 16u;
   uint32_t* tmem_slot_ptr = reinterpret_cast<uint32_t*>(smem + (tmem_slot - s_ring));
@@ -227,10 +244,12 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
 
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_x);
+    if (SILU) prefetch_tmap(&tm_y);
     if (LR) prefetch_tmap(&tm_pd);
     for (uint32_t s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), (LR ? 1 : 0) + NUM_QWARPS);
+      mbar_init(h_ready_bar(s), NUM_QWARPS);
     }
     mbar_init(lfull_bar, 1);
     mbar_init(final_bar, 1);
@@ -267,8 +286,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
         // Boxes are always delivered whole (zero fill past M and K); only
         // the smooth copy is cut to the chunks that exist.
         const uint32_t sm_bytes = p.smooth != nullptr ? nc * 128u : 0u;
-        mbar_arrive_expect_tx(full_bar(s), S::X_BYTES + S::PD_STAGE + sm_bytes);
+        mbar_arrive_expect_tx(full_bar(s), S::X_BYTES + S::Y_STAGE + S::PD_STAGE + sm_bytes);
         tma_load_3d(s_x(s), &tm_x, 0, mb * BM, kc0, full_bar(s));
+        if (SILU) tma_load_3d(s_y(s), &tm_y, 0, mb * BM, kc0, full_bar(s));
         if (LR) tma_load_3d(s_pd(s), &tm_pd, 0, kc0 * BKE, 0, full_bar(s));
         if (sm_bytes) bulk_load(s_sm(s), p.smooth + kc0 * BKE, sm_bytes, full_bar(s));
       }
@@ -291,7 +311,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
       for (int i = 0; i < nstages; ++i) {
         const uint32_t s = static_cast<uint32_t>(i) % STAGES;
         const uint32_t ph = (static_cast<uint32_t>(i) / STAGES) & 1u;
-        if (!svdq_wait(full_bar(s), ph, SITE_MMA)) {
+        // SILU: the MMA reads the formed silu(a) * b, after every quantizer
+        // warp wrote its part (which it did after the stage landed).
+        if (!svdq_wait(SILU ? h_ready_bar(s) : full_bar(s), ph, SITE_MMA)) {
           ok = false;
           break;
         }
@@ -348,6 +370,25 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x {64, M, K/
       // In a range's last stage the second chunk may be absent: those lanes
       // compute nothing but still take part in the shuffles below.
       const bool active = kc < c_end;
+      if constexpr (SILU) {
+        // x = silu(a) * b, written over a in the x slot (same swizzled
+        // places) for the MMA and for the quantizer reads below.
+        if (active) {
+#pragma unroll
+          for (int rr = 0; rr < S::ROWS_PER_THREAD; ++rr) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const uint32_t off = (hh ? xo1 : xo0) + rr * 64 * 128;
+              const uint4 a4 = lds_v4(s_x(s) + off), b4 = lds_v4(s_y(s) + off);
+              st_shared_v4(s_x(s) + off, silu_mul_bf16x2(a4.x, b4.x), silu_mul_bf16x2(a4.y, b4.y),
+                           silu_mul_bf16x2(a4.z, b4.z), silu_mul_bf16x2(a4.w, b4.w));
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(h_ready_bar(s));
+      }
       uint32_t sca = 0, scb = 0;
       if (active) {
         uint64_t nsm[8];

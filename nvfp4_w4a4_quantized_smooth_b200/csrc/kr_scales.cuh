@@ -16,6 +16,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "sm100_ptx.cuh"
+
 namespace svdq {
 namespace kr {
 
@@ -94,14 +96,7 @@ __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
     const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
     uint32_t wo[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float a0 = __uint_as_float(wa[j] << 16), a1 = __uint_as_float(wa[j] & 0xFFFF0000u);
-      const float b0 = __uint_as_float(wb[j] << 16), b1 = __uint_as_float(wb[j] & 0xFFFF0000u);
-      const float o0 = a0 / (1.0f + expf(-a0)) * b0;
-      const float o1 = a1 / (1.0f + expf(-a1)) * b1;
-      __nv_bfloat162 r = __floats2bfloat162_rn(o0, o1);
-      wo[j] = *reinterpret_cast<uint32_t*>(&r);
-    }
+    for (int j = 0; j < 4; ++j) wo[j] = silu_mul_bf16x2(wa[j], wb[j]);
     o4[i] = make_uint4(wo[0], wo[1], wo[2], wo[3]);
   }
   // tail
@@ -110,7 +105,7 @@ __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
   if (tail0 + tid < n) {
     const float av = __bfloat162float(a[tail0 + tid]);
     const float bv = __bfloat162float(b[tail0 + tid]);
-    out[tail0 + tid] = __float2bfloat16_rn(av / (1.0f + expf(-av)) * bv);
+    out[tail0 + tid] = __float2bfloat16_rn(silu_mul_f32(av, bv));
   }
 }
 

@@ -113,6 +113,24 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// ------------------------------------------------------------- SiLU * mul --
+// silu(a) * b = a / (1 + exp(-a)) * b in fp32 (the DiT feed-forward's gated
+// activation, w2's input), with CUDA's fast exponential and division
+// intrinsics (a few ulp of fp32, far below the bf16 rounding that follows).
+// One definition for every kernel that forms it, so that a fused and an
+// unfused path round to the same bf16.
+__device__ __forceinline__ float silu_mul_f32(float a, float b) {
+  return __fdividef(a, 1.0f + __expf(-a)) * b;
+}
+// Eight bf16 pairs (element 2i in the low half of word i) -> bf16 pairs of
+// silu(a) * b, nearest-even.
+__device__ __forceinline__ uint32_t silu_mul_bf16x2(uint32_t a, uint32_t b) {
+  const float lo = silu_mul_f32(__uint_as_float(a << 16), __uint_as_float(b << 16));
+  const float hi = silu_mul_f32(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u));
+  __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
 // ------------------------------------------------- dependent launches --
 // A kernel launched with programmatic stream serialization may start while
 // the previous kernel in the stream is still running.  griddep_wait blocks

@@ -54,18 +54,27 @@ int device_setup(DeviceInfo** out) {
       for (int& v : row) v = -1;
     if (d.sm100) {
       using namespace svdq;
-      if (cudaFuncSetAttribute(kq::quantize_act_kernel<64, true>,
+      if (cudaFuncSetAttribute(kq::quantize_act_kernel<64, true, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kq::Shape<64, true>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(kq::quantize_act_kernel<128, true>,
+          cudaFuncSetAttribute(kq::quantize_act_kernel<128, true, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kq::Shape<128, true>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(kq::quantize_act_kernel<64, false>,
+          cudaFuncSetAttribute(kq::quantize_act_kernel<64, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kq::Shape<64, false>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(kq::quantize_act_kernel<128, false>,
+          cudaFuncSetAttribute(kq::quantize_act_kernel<128, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kq::Shape<128, false>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kq::quantize_act_kernel<64, true, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kq::Shape<64, true, true>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kq::quantize_act_kernel<64, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kq::Shape<64, false, true>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kq::quantize_act_kernel<128, false, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kq::Shape<128, false, true>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(kg::w4a4_linear_kernel<true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kg::SMEM_BYTES) != cudaSuccess ||
@@ -156,8 +165,8 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const void* fn =
-      bm == 128 ? reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<128, true>)
-                : reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<64, true>);
+      bm == 128 ? reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<128, true, false>)
+                : reinterpret_cast<const void*>(svdq::kq::quantize_act_kernel<64, true, false>);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -174,10 +183,11 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
 // tile height that pads M the least, then to the taller tile (less
 // proj_down traffic per row), then to the smaller split.
 // If none fits (very large M), 128-row tiles without a split.
-void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out) {
+void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out, bool tall_ok = true) {
   const int chunks = K / svdq::kq::BKE;
-  int best_bm = 128, best_split = 1, best_ctas = -1, best_pad = 0;
+  int best_bm = tall_ok ? 128 : 64, best_split = 1, best_ctas = -1, best_pad = 0;
   for (int bm : {128, 64}) {
+    if (bm == 128 && !tall_ok) continue;
     const int m_tiles = (M + bm - 1) / bm;
     const int pad = m_tiles * bm - M;
     for (int split = 1; split <= svdq::kq::MAX_SPLIT && (split == 1 || 4 * split <= chunks);
@@ -294,17 +304,35 @@ int svdq_repack_weights(const uint8_t* wscales, int N, int K, void* wscales_tile
   return bad ? SVDQ_ERR_INVALID_ARG : SVDQ_OK;
 }
 
-int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* smooth,
-                      const uint16_t* proj_down, int R, uint8_t* qact, void* ascales_tiled,
-                      uint16_t* lowrank, void* stream) {
+}  // extern "C"
+
+namespace {
+
+using svdq::kq::quantize_act_kernel;
+using svdq::kq::Shape;
+
+// One launch of the activation kernel instance <BM, LR, SILU>.
+template <int BM, bool LR, bool SILU>
+cudaError_t launch_kq(cudaLaunchConfig_t& cfg, const CUtensorMap& tm_x, const CUtensorMap& tm_y,
+                      const CUtensorMap& tm_pd, const svdq::kq::Params& p) {
+  cfg.dynamicSmemBytes = Shape<BM, LR, SILU>::SMEM_BYTES;
+  return cudaLaunchKernelEx(&cfg, quantize_act_kernel<BM, LR, SILU>, tm_x, tm_y, tm_pd, p);
+}
+
+// Shared by svdq_quantize_act (b == NULL: the input is a) and
+// svdq_silu_mul_quantize_act (the input is silu(a) * b, formed on chip).
+int quantize_act_impl(const uint16_t* a, const uint16_t* b, int M, int K, int ld,
+                      const uint16_t* smooth, const uint16_t* proj_down, int R, uint8_t* qact,
+                      void* ascales_tiled, uint16_t* lowrank, void* stream) {
   const bool lr = R != 0;
-  if (!x || !qact || !ascales_tiled || (lr && (!proj_down || !lowrank)))
+  const bool silu = b != nullptr;
+  if (!a || !qact || !ascales_tiled || (lr && (!proj_down || !lowrank)))
     return SVDQ_ERR_INVALID_ARG;
-  if (M < 1 || K < 16 || K % 16 || ldx < K) return SVDQ_ERR_SHAPE;
+  if (M < 1 || K < 16 || K % 16 || ld < K) return SVDQ_ERR_SHAPE;
   if ((R != svdq::kq::R && R != 0) || K % 64) return SVDQ_ERR_UNSUPPORTED;
-  if (!aligned(x, 16) || (smooth && !aligned(smooth, 16)) || !aligned(qact, 16) ||
-      !aligned(ascales_tiled, 16) || (lr && (!aligned(proj_down, 16) || !aligned(lowrank, 16))) ||
-      ldx % 8)
+  if (!aligned(a, 16) || (silu && !aligned(b, 16)) || (smooth && !aligned(smooth, 16)) ||
+      !aligned(qact, 16) || !aligned(ascales_tiled, 16) ||
+      (lr && (!aligned(proj_down, 16) || !aligned(lowrank, 16))) || ld % 8)
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
   if (int st = device_setup(&d)) return st;
@@ -312,16 +340,21 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   const int chunks = K / svdq::kq::BKE;
   int bm = 0, split = 0;
   if (lr)
-    kq_plan(d, M, K, &bm, &split);
+    kq_plan(d, M, K, &bm, &split, /*tall_ok=*/!silu);
   else
     kq_plan_plain(d, M, K, &bm, &split);
   const int m_tiles = (M + bm - 1) / bm;
 
-  // x viewed as {64 k, M rows, K/64 chunks} and proj_down as {64 r, K,
-  // 2 halves of R}, so that one box carries a whole 128-k stage.
-  CUtensorMap tm_x, tm_pd;
-  if (make_tmap3(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, svdq::kq::BKE, M, chunks,
-                 static_cast<uint64_t>(ldx) * 2, svdq::kq::BKE * 2, svdq::kq::BKE, bm, 2))
+  // x (a, b) viewed as {64 k, M rows, K/64 chunks} and proj_down as {64 r,
+  // K, 2 halves of R}, so that one box carries a whole 128-k stage.
+  CUtensorMap tm_x, tm_y, tm_pd;
+  if (make_tmap3(&tm_x, a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, svdq::kq::BKE, M, chunks,
+                 static_cast<uint64_t>(ld) * 2, svdq::kq::BKE * 2, svdq::kq::BKE, bm, 2))
+    return SVDQ_ERR_CUDA;
+  if (!silu)
+    tm_y = tm_x;   // not read
+  else if (make_tmap3(&tm_y, b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, svdq::kq::BKE, M, chunks,
+                      static_cast<uint64_t>(ld) * 2, svdq::kq::BKE * 2, svdq::kq::BKE, bm, 2))
     return SVDQ_ERR_CUDA;
   if (!lr)
     tm_pd = tm_x;   // not read
@@ -343,10 +376,6 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(split, m_tiles, 1);
   cfg.blockDim = dim3(svdq::kq::NUM_THREADS, 1, 1);
-  using svdq::kq::Shape;
-  using svdq::kq::quantize_act_kernel;
-  cfg.dynamicSmemBytes = lr ? (bm == 128 ? Shape<128, true>::SMEM_BYTES : Shape<64, true>::SMEM_BYTES)
-                            : (bm == 128 ? Shape<128, false>::SMEM_BYTES : Shape<64, false>::SMEM_BYTES);
   cfg.stream = static_cast<cudaStream_t>(stream);
   // The K ranges of a tile form a cluster only when their L partials are
   // summed (low-rank branch).
@@ -360,14 +389,42 @@ int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* 
   cfg.attrs = attr;
   cfg.numAttrs = lr ? 2 : 1;
   cudaError_t e;
-  if (lr)
-    e = bm == 128 ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<128, true>, tm_x, tm_pd, p)
-                  : cudaLaunchKernelEx(&cfg, quantize_act_kernel<64, true>, tm_x, tm_pd, p);
-  else
-    e = bm == 128 ? cudaLaunchKernelEx(&cfg, quantize_act_kernel<128, false>, tm_x, tm_pd, p)
-                  : cudaLaunchKernelEx(&cfg, quantize_act_kernel<64, false>, tm_x, tm_pd, p);
+  if (silu) {
+    // (128-row tiles with the low-rank branch do not fit three stages.)
+    if (lr)
+      e = launch_kq<64, true, true>(cfg, tm_x, tm_y, tm_pd, p);
+    else
+      e = bm == 128 ? launch_kq<128, false, true>(cfg, tm_x, tm_y, tm_pd, p)
+                    : launch_kq<64, false, true>(cfg, tm_x, tm_y, tm_pd, p);
+  } else if (lr) {
+    e = bm == 128 ? launch_kq<128, true, false>(cfg, tm_x, tm_y, tm_pd, p)
+                  : launch_kq<64, true, false>(cfg, tm_x, tm_y, tm_pd, p);
+  } else {
+    e = bm == 128 ? launch_kq<128, false, false>(cfg, tm_x, tm_y, tm_pd, p)
+                  : launch_kq<64, false, false>(cfg, tm_x, tm_y, tm_pd, p);
+  }
   if (e != cudaSuccess) return SVDQ_ERR_CUDA;
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int svdq_quantize_act(const uint16_t* x, int M, int K, int ldx, const uint16_t* smooth,
+                      const uint16_t* proj_down, int R, uint8_t* qact, void* ascales_tiled,
+                      uint16_t* lowrank, void* stream) {
+  return quantize_act_impl(x, nullptr, M, K, ldx, smooth, proj_down, R, qact, ascales_tiled,
+                           lowrank, stream);
+}
+
+int svdq_silu_mul_quantize_act(const uint16_t* a, const uint16_t* b, int M, int K, int ld,
+                               const uint16_t* smooth, const uint16_t* proj_down, int R,
+                               uint8_t* qact, void* ascales_tiled, uint16_t* lowrank,
+                               void* stream) {
+  if (!b) return SVDQ_ERR_INVALID_ARG;
+  return quantize_act_impl(a, b, M, K, ld, smooth, proj_down, R, qact, ascales_tiled, lowrank,
+                           stream);
 }
 
 int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint16_t* lowrank,

@@ -29,7 +29,7 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 6
+ABI_VERSION = 7
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
 
@@ -46,6 +46,7 @@ SIGNATURES = {
     "svdq_repack_weights": (_I, [_P, _I, _I, _P, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
     "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
+    "svdq_silu_mul_quantize_act": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
     "svdq_quantize_plan": (_I, [_I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "svdq_unpack_scales": (_I, [_P, _I, _I, _I, _P, _P]),
     "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
@@ -167,6 +168,41 @@ def quantize_act(x: torch.Tensor, smooth: Optional[torch.Tensor],
                                   _ptr(qact), _ptr(ascales_tiled), _ptr(lowrank if R else None),
                                   _stream(stream)),
            "svdq_quantize_act")
+    return qact, ascales_tiled, (lowrank if R else None)
+
+
+def silu_mul_quantize_act(a: torch.Tensor, b: torch.Tensor, smooth: Optional[torch.Tensor],
+                          proj_down: Optional[torch.Tensor],
+                          qact: Optional[torch.Tensor] = None,
+                          ascales_tiled: Optional[torch.Tensor] = None,
+                          lowrank: Optional[torch.Tensor] = None, stream=None):
+    """quantize_act of x = silu(a) * b (the w2 input of a DiT feed-forward
+    block), formed on the device without writing x -> (qact, ascales_tiled,
+    lowrank)."""
+    _need(a, torch.bfloat16, "a", 2)
+    _need(b, torch.bfloat16, "b", 2)
+    if a.shape != b.shape or a.stride() != b.stride() or a.stride(1) != 1:
+        raise ValueError("a and b must have the same shape and strides, unit stride along K")
+    if smooth is not None:
+        _need(smooth, torch.bfloat16, "smooth", 1)
+        smooth = smooth.contiguous()
+    if proj_down is not None:
+        _need(proj_down, torch.bfloat16, "proj_down", 2)
+        proj_down = proj_down.contiguous()
+    M, K = a.shape
+    R = 0 if proj_down is None else proj_down.shape[1]
+    dev = a.device
+    if qact is None:
+        qact = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    if ascales_tiled is None:
+        ascales_tiled = torch.empty(max(ascales_tiled_bytes(M, K), 1), dtype=torch.uint8,
+                                    device=dev)
+    if lowrank is None and R:
+        lowrank = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
+    _check(_lib.svdq_silu_mul_quantize_act(_ptr(a), _ptr(b), M, K, a.stride(0), _ptr(smooth),
+                                           _ptr(proj_down), R, _ptr(qact), _ptr(ascales_tiled),
+                                           _ptr(lowrank if R else None), _stream(stream)),
+           "svdq_silu_mul_quantize_act")
     return qact, ascales_tiled, (lowrank if R else None)
 
 

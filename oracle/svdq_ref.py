@@ -18,7 +18,7 @@ with the operand table of the same section:
     proj_down [K, R]    bf16      SVD residual, down factor (R = 128)
     proj_up   [N, R]    bf16      SVD residual, up factor
 
-Readings taken where the card is silent (each is listed in the design doc):
+Readings taken where the card is silent:
 
 * ``quant`` is dynamic NVFP4 quantization of each 16-element group along
   K: scale = e4m3(amax / 6), element = E2M1(v / scale), both rounded to

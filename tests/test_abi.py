@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(svdq):
 
 
 def test_abi_version_and_status_strings(svdq):
-    assert svdq.abi_version() == 6 == svdq.ABI_VERSION
+    assert svdq.abi_version() == 7 == svdq.ABI_VERSION
     for st in range(8):
         s = svdq._lib.svdq_status_string(st).decode()
         assert s.startswith("SVDQ")
@@ -112,6 +112,13 @@ def test_argument_checks_fail_before_any_device_work(svdq):
                                 256, 0, fake, 48, None) == svdq.SVDQ_ERR_UNSUPPORTED
     assert lib.svdq_w4a4_linear(fake, fake, None, fake, fake, fake, fake, None, None, 16, 64,
                                 256, 128, fake, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
+    # the fused w2 activation: b is required, the other checks as quantize_act
+    assert lib.svdq_silu_mul_quantize_act(fake, None, 16, 64, 64, fake, fake, 128, fake, fake,
+                                          fake, None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_silu_mul_quantize_act(fake, fake, 16, 64, 32, fake, fake, 128, fake, fake,
+                                          fake, None) == svdq.SVDQ_ERR_SHAPE
+    assert lib.svdq_silu_mul_quantize_act(fake, odd, 16, 64, 64, fake, fake, 128, fake, fake,
+                                          fake, None) == svdq.SVDQ_ERR_ALIGNMENT
     # scale unpack: only the two documented tile orders
     for kind in (-1, 2):
         assert lib.svdq_unpack_scales(fake, 16, 64, kind, fake, None) == svdq.SVDQ_ERR_INVALID_ARG

@@ -363,6 +363,59 @@ def test_full_size_ffn_chain():
     H.assert_y_close(r2["y"][rows], y_ref, "w2")
 
 
+@pytest.mark.parametrize("M,K,R", [(300, 512, 128), (64, 1024, 0), (1000, 2048, 128),
+                                   (4352, 10240, 128)])
+def test_fused_silu_mul_quantize(M, K, R):
+    # quantize_act of x = silu(a) * b, with x formed on chip: codes and
+    # scales identical to the unfused path (svdq_silu_mul, then
+    # svdq_quantize_act on its bf16 x), both equal to the oracle's on that
+    # x, and L within tolerance of the oracle.
+    s = H.svdq()
+    g = torch.Generator().manual_seed(M + K + R)
+    a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16).cuda()
+    b = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    sm = (torch.rand(K, generator=g) * 1.5 + 0.5).to(torch.bfloat16).cuda()
+    pd = (torch.randn(K, 128, generator=g) * 0.02).to(torch.bfloat16).cuda() if R else None
+    q1, a1, l1 = s.silu_mul_quantize_act(a, b, sm, pd)
+    h = s.silu_mul(a, b)
+    q2, a2, l2 = s.quantize_act(h, sm, pd)
+    s.check_device_error()
+    assert torch.equal(q1, q2)
+    asc1 = s.unpack_scales(a1, M, K).cpu()
+    assert torch.equal(asc1, s.unpack_scales(a2, M, K).cpu())
+    rows = H.sample_rows(M, 64, seed=K)
+    hc = h.cpu()
+    q_ref, a_ref = H.oracle_quant(hc[rows], sm.cpu())
+    H.assert_quant_exact(q1.cpu()[rows], asc1[rows], q_ref, a_ref, "fused silu quant")
+    if R:
+        L_ref = ref.lowrank_down(H.bits(hc[rows]), H.bits(pd.cpu()))
+        H.assert_lowrank_close(l1.cpu()[rows], L_ref, "fused silu L")
+    else:
+        assert l1 is None
+
+
+def test_full_size_ffn_chain_fused():
+    # w1, w3, then w2 with its input formed on chip from their outputs.
+    s = H.svdq()
+    names = ("ffn_w1_m4352_k3840_n10240", "ffn_w3_m4352_k3840_n10240", "ffn_w2_m4352_k10240_n3840")
+    L1, L3, L2 = (synth.make_layer(*synth.WORKLOADS[n], seed=synth.workload_seed(n)) for n in names)
+    L3.x = L1.x
+    r1, r3 = H.gpu_layer(L1), H.gpu_layer(L3)
+    y1, y3 = r1["y"].cuda(), r3["y"].cuda()
+    d = H.to_dev(L2)
+    wt = s.repack_weights(d["wscales"])
+    qa, asc, lr = s.silu_mul_quantize_act(y1, y3, d["smooth"], d["proj_down"])
+    y = s.w4a4_linear(qa, asc, lr, d["qweight"], wt, d["wcscales"], d["wtscale"], d["proj_up"],
+                      d["bias"])
+    s.check_device_error()
+    h = s.silu_mul(y1, y3).cpu()
+    rows = H.sample_rows(L2.M, 24, seed=9)
+    y_ref, q_ref, a_ref, _ = H.oracle_y(L2, rows=rows, x=h)
+    H.assert_quant_exact(qa.cpu()[rows], s.unpack_scales(asc, L2.M, L2.K).cpu()[rows], q_ref,
+                         a_ref, "fused w2 quant")
+    H.assert_y_close(y.cpu()[rows], y_ref, "fused w2")
+
+
 def test_silu_mul_tail_and_values():
     s = H.svdq()
     g = torch.Generator().manual_seed(3)
