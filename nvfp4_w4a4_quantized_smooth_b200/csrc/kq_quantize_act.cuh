@@ -370,31 +370,16 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       // In a range's last stage the second chunk may be absent: those lanes
       // compute nothing but still take part in the shuffles below.
       const bool active = kc < c_end;
-      if constexpr (SILU) {
-        // x = silu(a) * b, written over a in the x slot (same swizzled
-        // places) for the MMA and for the quantizer reads below.
-        if (active) {
-#pragma unroll
-          for (int rr = 0; rr < S::ROWS_PER_THREAD; ++rr) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const uint32_t off = (hh ? xo1 : xo0) + rr * 64 * 128;
-              const uint4 a4 = lds_v4(s_x(s) + off), b4 = lds_v4(s_y(s) + off);
-              st_shared_v4(s_x(s) + off, silu_mul_bf16x2(a4.x, b4.x), silu_mul_bf16x2(a4.y, b4.y),
-                           silu_mul_bf16x2(a4.z, b4.z), silu_mul_bf16x2(a4.w, b4.w));
-            }
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(h_ready_bar(s));
-      }
-      uint32_t sca = 0, scb = 0;
+      // This thread's inputs -> registers: smooth (negated, packed fp32
+      // pairs) and x for its one or two rows.
+      uint64_t nsm[8];
+      uint32_t xv[S::ROWS_PER_THREAD][8];
+      uint32_t got = 0;   // depends on every value read from the stage
       if (active) {
-        uint64_t nsm[8];
         if (p.smooth != nullptr) {
           const uint4 sa = lds_v4(s_sm(s) + cg * 32);
           const uint4 sb = lds_v4(s_sm(s) + cg * 32 + 16);
+          got ^= sa.x ^ sa.y ^ sa.z ^ sa.w ^ sb.x ^ sb.y ^ sb.z ^ sb.w;
           const uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
           for (int j = 0; j < 8; ++j) nsm[j] = bf16x2_to_pk(sw[j] ^ 0x80008000u);
@@ -403,25 +388,53 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
 #pragma unroll
           for (int j = 0; j < 8; ++j) nsm[j] = pk(-1.0f, -1.0f);
         }
-        const uint32_t xs = s_x(s);
-        const uint4 a0 = lds_v4(xs + xo0), a1 = lds_v4(xs + xo1);
-        const uint32_t xa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+        for (int rr = 0; rr < S::ROWS_PER_THREAD; ++rr) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t off = (hh ? xo1 : xo0) + rr * 64 * 128;
+            uint4 v4 = lds_v4(s_x(s) + off);
+            got ^= v4.x ^ v4.y ^ v4.z ^ v4.w;
+            if constexpr (SILU) {
+              // x = silu(a) * b, written over a in the x slot (same
+              // swizzled places) for the MMA
+              const uint4 b4 = lds_v4(s_y(s) + off);
+              got ^= b4.x ^ b4.y ^ b4.z ^ b4.w;
+              v4 = make_uint4(silu_mul_bf16x2(v4.x, b4.x), silu_mul_bf16x2(v4.y, b4.y),
+                              silu_mul_bf16x2(v4.z, b4.z), silu_mul_bf16x2(v4.w, b4.w));
+              st_shared_v4(s_x(s) + off, v4.x, v4.y, v4.z, v4.w);
+            }
+            xv[rr][4 * hh] = v4.x;
+            xv[rr][4 * hh + 1] = v4.y;
+            xv[rr][4 * hh + 2] = v4.z;
+            xv[rr][4 * hh + 3] = v4.w;
+          }
+        }
+      }
+      if constexpr (SILU) {
+        // x is in place for the MMA, and every lane's reads of the stage
+        // have returned (the asm needs their values) and are ordered before
+        // the async-proxy copy that refills it: the stage is released now,
+        // so the arithmetic below overlaps that copy.
+        asm volatile("" ::"r"(got) : "memory");
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(h_ready_bar(s));
+          mbar_arrive(empty_bar(s));
+        }
+      }
+      uint32_t sca = 0, scb = 0;
+      if (active) {
+        const uint64_t ca = quantize_group(xv[0], nsm, sca);
+        if (m0 < p.M)
+          *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
+              make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
         if constexpr (S::ROWS_PER_THREAD == 2) {
-          const uint4 b0 = lds_v4(xs + xo0 + 64 * 128), b1 = lds_v4(xs + xo1 + 64 * 128);
-          const uint32_t xb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-          const uint64_t ca = quantize_group(xa, nsm, sca);
-          const uint64_t cb = quantize_group(xb, nsm, scb);
-          if (m0 < p.M)
-            *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
-                make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
+          const uint64_t cb = quantize_group(xv[S::ROWS_PER_THREAD - 1], nsm, scb);
           if (m1 < p.M)
             *reinterpret_cast<uint2*>(q1_row + kc * (BKE / 2)) =
                 make_uint2(static_cast<uint32_t>(cb), static_cast<uint32_t>(cb >> 32));
-        } else {
-          const uint64_t ca = quantize_group(xa, nsm, sca);
-          if (m0 < p.M)
-            *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
-                make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
         }
       }
       // Lanes 4j..4j+3 hold one row's four groups of one chunk.
@@ -443,8 +456,11 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
         if (active && g == 0 && m1 >= static_cast<int>(gridDim.y) * BM && m1 < rows_pad)
           *reinterpret_cast<uint32_t*>(sc1 + static_cast<size_t>(kc) * 512) = 0u;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar(s));
+      if constexpr (!SILU) {
+        // the stage's values have all been used: release it
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+      }
     }
     if (LR) l_ready = ok && __all_sync(0xFFFFFFFFu, svdq_wait(lfull_bar, 0, SITE_LFULL));
   }
