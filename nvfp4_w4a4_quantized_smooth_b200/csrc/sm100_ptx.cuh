@@ -200,19 +200,6 @@ __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-// Contiguous bulk copy shared (this CTA) -> global, tracked by the issuing
-// thread's bulk async-group; 16-byte aligned, size % 16 == 0.
-__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
-               "r"(bytes)
-               : "memory");
-}
-// Orders this thread's global-memory accesses through the generic proxy
-// with those through the async proxy (bulk copies).
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // Contiguous bulk copy global -> shared; 16-byte aligned, size % 16 == 0.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -281,13 +268,6 @@ __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint
       "p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
-}
-
-// Copy 32 rows x 16 bytes of shared memory (one 512-byte scale block) into
-// TMEM lanes 0..31 of 4 columns, replicated into all four lane quarters.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
 }
 
 // Load 32 consecutive 32-bit TMEM columns of this warp's lane quarter: each
@@ -377,13 +357,7 @@ __host__ __device__ constexpr uint32_t idesc_nvfp4(uint32_t M, uint32_t N) {
          | ((M >> 4) << 24);        // M / 16
 }
 
-
 // --------------------------------------------------------------- cluster --
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                "barrier.cluster.wait.acquire.aligned;" ::

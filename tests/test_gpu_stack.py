@@ -6,8 +6,9 @@ Blocks 0, 14 and 29: 16 sampled rows of every linear, all columns, with
 their codes and scales bit-exact; block 0's whole input is also quantized
 and compared code for code.  Every other linear: 8 sampled rows x 64
 sampled columns of y, and the codes and scales of those rows.  The w2
-input is silu(y_w1) * y_w3 from the GPU's own bf16 outputs, and its oracle
-takes that same input, so errors do not compound.
+input is silu(y_w1) * y_w3 of the GPU's own bf16 outputs, formed on chip by
+the fused activation kernel; its oracle takes that same input (formed by
+svdq_silu_mul, bit for bit the same), so errors do not compound.
 """
 
 import numpy as np
@@ -48,8 +49,15 @@ def test_dit_stack_30_blocks():
             w = s.PreparedWeights(L.qweight.cuda(), L.wscales.cuda(), L.wcscales.cuda(),
                                   L.wtscale.cuda(), L.smooth.cuda(), L.proj_down.cuda(),
                                   L.proj_up.cuda(), L.bias.cuda())
-            x_in = h if name == "w2" else xd
-            qa, asc, lr = s.quantize_act(x_in, w.smooth, w.proj_down)
+            if name == "w2":
+                # w2's input formed on chip from w1's and w3's outputs; the
+                # oracle takes the same x, formed by svdq_silu_mul
+                x_in = h
+                qa, asc, lr = s.silu_mul_quantize_act(y13["w1"], y13["w3"], w.smooth,
+                                                      w.proj_down)
+            else:
+                x_in = xd
+                qa, asc, lr = s.quantize_act(x_in, w.smooth, w.proj_down)
             y = s.w4a4_linear(qa, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
                               w.proj_up, w.bias)
             s.check_device_error()
