@@ -425,3 +425,50 @@ def test_silu_mul_tail_and_values():
         out = s.silu_mul(a.cuda(), b.cuda()).cpu()
         want = (a.float() * torch.sigmoid(a.float()) * b.float())
         assert ((out.float() - want).abs() <= 2 ** -7 * want.abs() + 1e-6).all(), n
+
+
+# ------------------------------------------------ seeded shape sweep ---
+
+def _sweep_shapes(n, seed):
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        M = int(rng.integers(1, 700))
+        K = 256 * int(rng.integers(1, 9))
+        N = 32 * int(rng.integers(1, 33))
+        out.append((M, K, N))
+    return out
+
+
+@pytest.mark.parametrize("M,K,N", _sweep_shapes(12, 2026))
+def test_shape_sweep_all_paths(M, K, N):
+    # Seeded shapes (ragged M, N and several K) through every path: the
+    # layer, the layer without the low-rank branch (with and without
+    # smooth), and w2's activation formed on chip; each against the oracle,
+    # and each repeated bit for bit.
+    s = H.svdq()
+    L = synth.make_layer(M, K, N, seed=M * 7 + K + N)
+    r = H.gpu_layer(L)
+    y_ref, q_ref, a_ref, L_ref = H.oracle_y(L)
+    H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, f"layer {M}x{K}x{N}")
+    H.assert_y_close(r["y"], y_ref, f"layer {M}x{K}x{N}")
+    H.assert_lowrank_close(r["lowrank"], L_ref, f"layer {M}x{K}x{N}")
+    again = H.gpu_layer(L)
+    assert torch.equal(again["y"].view(torch.int16), r["y"].view(torch.int16))
+    for with_smooth in (False, True):
+        p = H.gpu_plain_layer(L, with_smooth)
+        yp, qp, ap = H.oracle_plain_y(L, with_smooth)
+        H.assert_quant_exact(p["qact"], p["ascales"], qp, ap, f"plain {M}x{K}x{N}")
+        H.assert_y_close(p["y"], yp, f"plain {M}x{K}x{N}")
+    g = torch.Generator().manual_seed(M + N)
+    a = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    b = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    d = H.to_dev(L)
+    q1, a1, l1 = s.silu_mul_quantize_act(a, b, d["smooth"], d["proj_down"])
+    h = s.silu_mul(a, b)
+    q2, a2, l2 = s.quantize_act(h, d["smooth"], d["proj_down"])
+    s.check_device_error()
+    assert torch.equal(q1, q2)
+    assert torch.equal(s.unpack_scales(a1, M, K).cpu(), s.unpack_scales(a2, M, K).cpu())
+    Lh = ref.lowrank_down(H.bits(h.cpu()), H.bits(L.proj_down))
+    H.assert_lowrank_close(l1.cpu(), Lh, f"fused L {M}x{K}")
