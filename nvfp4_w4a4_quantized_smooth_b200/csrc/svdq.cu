@@ -13,6 +13,7 @@
 #include "sm100_ptx.cuh"
 #include "kq_quantize_act.cuh"
 #include "kg_w4a4_linear.cuh"
+#include "ks_w4a4_linear_small.cuh"
 #include "kr_scales.cuh"
 
 namespace {
@@ -80,7 +81,13 @@ int device_setup(DeviceInfo** out) {
                                kg::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(kg::w4a4_linear_kernel<false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kg::SMEM_BYTES) != cudaSuccess)
+                               kg::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(ks::w4a4_linear_small_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ks::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(ks::w4a4_linear_small_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ks::SMEM_BYTES) != cudaSuccess)
         return SVDQ_ERR_CUDA;
     }
     if (g_encode == nullptr) {
@@ -117,16 +124,17 @@ int make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t
 
 // 3-D tensor map: dims {d0 (contiguous), d1, d2} with byte strides s1, s2
 // for dims 1 and 2 (any order; the views used here interleave them), box
-// {b0, b1, b2}, landing in shared memory as [b2][b1][b0]; 128-byte swizzle,
-// zero fill outside the tensor.
+// {b0, b1, b2}, landing in shared memory as [b2][b1][b0]; 128-byte swizzle
+// (or none), zero fill outside the tensor.
 int make_tmap3(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t d0, uint64_t d1,
-               uint64_t d2, uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+               uint64_t d2, uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {s1, s2};
   cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
@@ -134,6 +142,68 @@ int make_tmap3(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_
 int launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+// The GEMM for M <= 64 tokens (ks_w4a4_linear_small.cuh): weights as the
+// 128-row MMA operand, one CTA per 128 weight rows.  Arguments as checked
+// by svdq_w4a4_linear.
+int launch_small(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
+                 const uint16_t* lowrank, const uint8_t* qweight, const void* wscales_tiled,
+                 const uint16_t* wcscales, const uint16_t* wtscale, const uint16_t* proj_up,
+                 const uint16_t* bias, int M, int N, int K, int R, uint16_t* y, int ldy,
+                 void* stream) {
+  namespace ks = svdq::ks;
+  const bool lr = R != 0;
+  const uint64_t kb = static_cast<uint64_t>(K) / 2;
+  const uint64_t n_tiles256 = (static_cast<uint64_t>(N) + 255) / 256;
+  const uint64_t kblocks = static_cast<uint64_t>(K) / 64;
+  CUtensorMap tm_w, tm_x, tm_sw, tm_p, tm_l, tm_y;
+  // Repacked weight scales: per 256-row tile and 64-k block, 1024 bytes
+  // (rows 0..127, then 128..255), viewed as u32 {128, half, tile * kblocks}.
+  if (make_tmap(&tm_w, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, N, kb, ks::BK_BYTES, ks::BMW) ||
+      make_tmap(&tm_x, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, ks::BK_BYTES, ks::NT) ||
+      make_tmap3(&tm_sw, wscales_tiled, CU_TENSOR_MAP_DATA_TYPE_UINT32, 128, 2,
+                 n_tiles256 * kblocks, 512, 1024, 128, 1, 4, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      make_tmap(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(ldy) * 2,
+                ks::BMW, ks::NT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SVDQ_ERR_CUDA;
+  if (!lr) {
+    tm_p = tm_w;   // not read
+    tm_l = tm_x;
+  } else if (make_tmap(&tm_p, proj_up, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, N,
+                       static_cast<uint64_t>(R) * 2, 64, ks::BMW) ||
+             make_tmap(&tm_l, lowrank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, M,
+                       static_cast<uint64_t>(R) * 2, 64, ks::NT)) {
+    return SVDQ_ERR_CUDA;
+  }
+  ks::Params p;
+  p.ascales_tiled = static_cast<const uint8_t*>(ascales_tiled);
+  p.wcscales = reinterpret_cast<const __nv_bfloat16*>(wcscales);
+  p.wtscale = reinterpret_cast<const __nv_bfloat16*>(wtscale);
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_tiles = (N + ks::BMW - 1) / ks::BMW;
+  const int grid = p.n_tiles < d->num_sms ? p.n_tiles : d->num_sms;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(ks::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = ks::SMEM_BYTES;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e =
+      lr ? cudaLaunchKernelEx(&cfg, ks::w4a4_linear_small_kernel<true>, tm_w, tm_x, tm_sw, tm_p,
+                              tm_l, tm_y, p)
+         : cudaLaunchKernelEx(&cfg, ks::w4a4_linear_small_kernel<false>, tm_w, tm_x, tm_sw, tm_p,
+                              tm_l, tm_y, p);
+  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
+  return launch_status();
 }
 
 int grid_for(size_t work, int threads, int num_sms) {
@@ -446,6 +516,9 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   if (int st = device_setup(&d)) return st;
 
   const uint64_t kb = static_cast<uint64_t>(K) / 2;
+  if (M <= svdq::ks::NT)
+    return launch_small(d, qact, ascales_tiled, lowrank, qweight, wscales_tiled, wcscales,
+                        wtscale, proj_up, bias, M, N, K, R, y, ldy, stream);
   CUtensorMap tm_a, tm_b, tm_l, tm_p, tm_y;
   if (make_tmap(&tm_a, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, svdq::kg::BK_BYTES,
                 svdq::kg::BM) ||

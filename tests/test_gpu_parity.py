@@ -472,3 +472,24 @@ def test_shape_sweep_all_paths(M, K, N):
     assert torch.equal(s.unpack_scales(a1, M, K).cpu(), s.unpack_scales(a2, M, K).cpu())
     Lh = ref.lowrank_down(H.bits(h.cpu()), H.bits(L.proj_down))
     H.assert_lowrank_close(l1.cpu(), Lh, f"fused L {M}x{K}")
+
+
+# ------------------------------------------------ few tokens (M <= 64) ---
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 128), (7, 10240, 3840), (33, 1024, 416), (64, 512, 384),
+                                   (64, 768, 11520), (64, 2048, 20480)])
+def test_small_m_transposed_gemm(M, K, N):
+    # M <= 64 runs the transposed GEMM (weights as the 128-row operand):
+    # one token, ragged M and N, a long K, more 128-column tiles than SMs
+    # (the persistent loop) -- with and without the low-rank branch,
+    # against the oracle, and repeated bit for bit.
+    L = synth.make_layer(M, K, N, seed=M * 3 + K + N)
+    r = H.gpu_layer(L)
+    y_ref, q_ref, a_ref, L_ref = H.oracle_y(L)
+    H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, f"{M}x{K}x{N}")
+    H.assert_y_close(r["y"], y_ref, f"{M}x{K}x{N}")
+    again = H.gpu_layer(L)
+    assert torch.equal(again["y"].view(torch.int16), r["y"].view(torch.int16))
+    p = H.gpu_plain_layer(L, True)
+    yp, _, _ = H.oracle_plain_y(L, True)
+    H.assert_y_close(p["y"], yp, f"plain {M}x{K}x{N}")
