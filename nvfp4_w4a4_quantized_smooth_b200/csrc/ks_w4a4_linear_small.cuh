@@ -7,9 +7,15 @@
 //   acc^T[n, m] = sum_k e2m1(qw[n,k]) sw[k/16,n] e2m1(qa[m,k]) sa[m,k/16]
 // The weights are the MMA's 128-row A operand and the (at most 64) tokens
 // its N = 64 operand, so N / 128 CTAs share the weight stream, each over
-// the whole K range (a 128-token x 256-column tile would leave N / 256 CTAs
-// for it).  One CTA per 128 weight rows; persistent when there are more
-// such tiles than SMs.
+// its K range (a 128-token x 256-column tile would leave N / 256 CTAs for
+// it).  One CTA per 128 weight rows and K range: with `split` > 1 the K
+// steps of a tile are divided among the `split` CTAs of a thread-block
+// cluster, each of which keeps its fp32 partial tile (and its own copy of
+// the low-rank tile) in shared memory; after a cluster barrier rank r sums
+// the partials of rows [r 128 / split, (r + 1) 128 / split) in rank order
+// through distributed shared memory (deterministic), applies the epilogue
+// and stores those columns of y.  With `split` = 1 a CTA covers the whole
+// K range and loops over tiles when there are more than SMs.
 //
 // Roles (192 threads):
 //   warp 0      producer (one thread): a ring of SLOTS slots, one K step of
@@ -18,20 +24,21 @@
 //               512-byte scale blocks of the tile's 128 weight rows (one 3-D
 //               box out of the 256-row tile order of the repacked weight
 //               scales) and the four scale blocks of the tokens (one bulk
-//               copy).  After a tile's K steps two more slots carry the
-//               low-rank halves (proj_up half in the weight place, L half in
-//               the token place).
+//               copy).  A tile's first two slots carry the low-rank halves
+//               (proj_up half in the weight place, L half in the token
+//               place), so that their latency overlaps the K steps.
 //   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma
-//               kind::mxf4nvf4 block16, M = 128, N = 64, K = 64, then
-//               kind::f16 (bf16, K = 16) for proj_up @ L^T into a second
-//               accumulator.
+//               kind::f16 (bf16, K = 16) for proj_up @ L^T into the low-rank
+//               accumulator, then kind::mxf4nvf4 block16, M = 128, N = 64,
+//               K = 64 into the main one.
 //   warps 2..5  one per TMEM lane quarter.  During the K loop: slot s's
 //               scale blocks -> TMEM scale slot s (tcgen05.st, each block
 //               replicated in the four lane quarters, as the MMA reads it).
 //               After it, the epilogue: TMEM -> registers, fp32
 //               acc * wtscale * wcscales + lr + bias -> bf16, transposed
 //               into a [64 tokens][128 columns] shared buffer, then one TMA
-//               tensor store, which clips the M and N edges.
+//               tensor store, which clips the M and N edges (split > 1:
+//               both accumulators -> shared memory for the cluster sum).
 // TMEM (512 columns): accumulator [0, 64), low-rank accumulator [64, 128),
 // scale slot s at [128 + 32 s, 160 + 32 s): weight scales (4 MMAs x 4
 // columns), then token scales (4 x 4).
@@ -85,8 +92,10 @@ struct Params {
   const __nv_bfloat16* wcscales;
   const __nv_bfloat16* wtscale;
   const __nv_bfloat16* bias;         // may be null
-  int M, N, K;
+  __nv_bfloat16* y;                  // [M, ldy], written directly when split > 1
+  int M, N, K, ldy;
   int n_tiles;                       // 128-row weight tiles
+  int split;                         // K ranges per tile = cluster size (1, 2, 4, 8)
 };
 
 // LR: the layer has the low-rank branch (R = 128); without it (R = 0) a
@@ -109,6 +118,11 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
   auto s_b = [&](uint32_t s) { return s_ring + s * SLOT_BYTES + A_BYTES; };
   auto s_sf = [&](uint32_t s) { return s_ring + s * SLOT_BYTES + A_BYTES + B_BYTES; };
   const uint32_t s_out = s_ring + RING_BYTES;
+  // After the last MMA (split > 1): this rank's partial and low-rank tiles,
+  // [64 tokens][128 columns] fp32 each, over the first two ring slots.
+  const uint32_t s_part = s_ring;
+  const uint32_t s_lrt = s_ring + NT * BMW * 4;
+  static_assert(2 * NT * BMW * 4 <= RING_BYTES, "partial tiles fit the ring");
   const uint32_t s_bar = s_out + OUT_BYTES;
   // barriers: slot full (TMA bytes), slot scales in TMEM, slot free
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
@@ -155,15 +169,22 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
   griddep_launch_dependents();
 
   const int num_k = p.K / BK;                  // K steps per tile
-  const int uses = num_k + (LR ? 2 : 0);       // ring slots per tile
   const int kblocks = p.K / 64;                // 512-byte scale blocks per 128 rows
+  const int split = p.split;
+  const int rank = split > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int k0 = num_k * rank / split;         // this CTA's K steps [k0, k0 + nk)
+  const int nk = num_k * (rank + 1) / split - k0;
+  const int lr_uses = LR ? 2 : 0;
+  const int uses = lr_uses + nk;               // ring slots per tile
+  const int tile0 = static_cast<int>(blockIdx.x) / split;
+  const int tile_step = static_cast<int>(gridDim.x) / split;
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ producer --
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+      for (int t = tile0; t < p.n_tiles && ok; t += tile_step) {
         for (int st = 0; st < uses; ++st, ++it) {
           const uint32_t s = it % SLOTS;
           const uint32_t ph = (it / SLOTS) & 1u;
@@ -171,19 +192,20 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
             ok = false;
             break;
           }
-          if (st < num_k) {
-            mbar_arrive_expect_tx(full_bar(s), SLOT_BYTES);
-            tma_load_2d(s_a(s), &tm_w, st * BK_BYTES, t * BMW, full_bar(s));
-            tma_load_2d(s_b(s), &tm_x, st * BK_BYTES, 0, full_bar(s));
-            // weight rows [128 t, 128 t + 128) = half (t & 1) of 256-row tile t / 2
-            tma_load_3d(s_sf(s), &tm_sw, 0, t & 1, (t >> 1) * kblocks + 4 * st, full_bar(s));
-            bulk_load(s_sf(s) + SFA_BYTES, p.ascales_tiled + static_cast<size_t>(4 * st) * 512,
-                      SFB_BYTES, full_bar(s));
-          } else {
-            const int hr = st - num_k;           // which 64-wide half of R
+          if (st < lr_uses) {
+            const int hr = st;                   // which 64-wide half of R
             mbar_arrive_expect_tx(full_bar(s), LR_A_BYTES + LR_B_BYTES);
             tma_load_2d(s_a(s), &tm_p, hr * 64, t * BMW, full_bar(s));
             tma_load_2d(s_b(s), &tm_l, hr * 64, 0, full_bar(s));
+          } else {
+            const int kk = k0 + st - lr_uses;    // K step
+            mbar_arrive_expect_tx(full_bar(s), SLOT_BYTES);
+            tma_load_2d(s_a(s), &tm_w, kk * BK_BYTES, t * BMW, full_bar(s));
+            tma_load_2d(s_b(s), &tm_x, kk * BK_BYTES, 0, full_bar(s));
+            // weight rows [128 t, 128 t + 128) = half (t & 1) of 256-row tile t / 2
+            tma_load_3d(s_sf(s), &tm_sw, 0, t & 1, (t >> 1) * kblocks + 4 * kk, full_bar(s));
+            bulk_load(s_sf(s) + SFA_BYTES, p.ascales_tiled + static_cast<size_t>(4 * kk) * 512,
+                      SFB_BYTES, full_bar(s));
           }
         }
       }
@@ -203,10 +225,29 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
       const uint32_t idesc_lr = idesc_bf16_f32(BMW, NT, 0, 0);
       uint32_t it = 0, tc = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++tc) {
+      for (int t = tile0; t < p.n_tiles && ok; t += tile_step, ++tc) {
         if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_MMA_TE)) break;
         tc_fence_after();
-        for (int st = 0; st < num_k; ++st, ++it) {
+        if (LR) {
+          // The low-rank accumulator has its own columns.
+          for (int hr = 0; hr < 2 && ok; ++hr, ++it) {
+            const uint32_t s = it % SLOTS;
+            const uint32_t ph = (it / SLOTS) & 1u;
+            if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16(tmem_base + TM_LR, smem_desc(s_a(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B),
+                      smem_desc(s_b(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B), idesc_lr,
+                      (hr | kk) != 0 ? 1u : 0u);
+            tc_commit(empty_bar(s));
+          }
+          if (!ok) break;
+        }
+        for (int st = 0; st < nk; ++st, ++it) {
           const uint32_t s = it % SLOTS;
           const uint32_t ph = (it / SLOTS) & 1u;
           if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL) ||
@@ -226,25 +267,6 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
           tc_commit(empty_bar(s));
         }
         if (!ok) break;
-        if (LR) {
-          // The low-rank accumulator has its own columns: no drain needed.
-          for (int hr = 0; hr < 2 && ok; ++hr, ++it) {
-            const uint32_t s = it % SLOTS;
-            const uint32_t ph = (it / SLOTS) & 1u;
-            if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16(tmem_base + TM_LR, smem_desc(s_a(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B),
-                      smem_desc(s_b(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B), idesc_lr,
-                      (hr | kk) != 0 ? 1u : 0u);
-            tc_commit(empty_bar(s));
-          }
-          if (!ok) break;
-        }
         tc_commit(tmem_full_bar);
       }
       // Every MMA this thread issued completes before TMEM is released.
@@ -259,7 +281,7 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
     const int n_local = q * 32 + lane;   // this thread's weight row in the tile
     uint32_t it = 0, tc = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++tc) {
+    for (int t = tile0; t < p.n_tiles; t += tile_step, ++tc) {
       // Scale blocks of each K step -> this quarter's lanes of TMEM slot s
       // (block b at columns 4 b .. 4 b + 3: weight blocks 0..3, token
       // blocks 4..7).  The slot's previous MMAs have completed: the
@@ -271,7 +293,7 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
         const uint32_t ph = (it / SLOTS) & 1u;
         if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(full_bar(s), ph, SITE_SF_FULL));
         if (!ok) continue;
-        if (st < num_k) {
+        if (st >= lr_uses) {
           tc_fence_after();
           const uint32_t src = s_sf(s) + 16 * lane;
           const uint32_t dst = lane_base + TM_SF + TM_SF_SLOT * s;
@@ -297,7 +319,30 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
         if (p.bias != nullptr) bs = __bfloat162float(p.bias[n]);
       }
       if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI));
-      if (ok) {
+      if (ok && split > 1) {
+        // This rank's partial tile and its low-rank tile -> shared memory
+        // ([token][column] fp32 at the start of the ring, which no MMA or
+        // copy uses any more), for the cluster sum after the role loops.
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < NT / 16; ++c) {
+          uint32_t acc[16], lr[16];
+          tmem_ld_32x32b_x16(lane_base + TM_ACC + 16 * c, acc);
+          if (LR) {
+            tmem_ld_32x32b_x16(lane_base + TM_LR + 16 * c, lr);
+          } else {
+#pragma unroll
+            for (int z = 0; z < 16; ++z) lr[z] = 0u;   // +0.0f
+          }
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint32_t off = static_cast<uint32_t>((16 * c + i) * BMW + n_local) * 4u;
+            st_shared_f32(s_part + off, __uint_as_float(acc[i]));
+            st_shared_f32(s_lrt + off, __uint_as_float(lr[i]));
+          }
+        }
+      } else if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < NT / 16; ++c) {
@@ -327,7 +372,7 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
       }
       named_bar_sync(1, 32 * NUM_EPI_WARPS);
       if (warp == EPI_WARP0 && lane == 0) {
-        if (ok) {
+        if (ok && split == 1) {
           tma_store_2d(&tm_y, s_out, t * BMW, 0);
           bulk_commit_group();
         }
@@ -336,6 +381,57 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
       named_bar_sync(1, 32 * NUM_EPI_WARPS);
     }
     if (warp == EPI_WARP0 && lane == 0) bulk_wait_group0();
+  }
+
+  if (split > 1) {
+    // ------------------------------------------------- cluster K sum --
+    // Every thread of every rank takes both cluster barriers.  Rank r sums
+    // rows [r R0, (r + 1) R0) of the partial tiles of all ranks in rank
+    // order; a unit is 4 consecutive rows of one token (a float4 of each
+    // rank's [token][column] tile), so that a warp reads and writes whole
+    // 16-byte pieces.  The low-rank tile is this rank's own copy.
+    __syncwarp();
+    cluster_sync_all();
+    if (warp >= EPI_WARP0 && !error_raised()) {
+      const int et = static_cast<int>(threadIdx.x) - 32 * EPI_WARP0;   // 0..127
+      const int r0 = BMW / split;                  // rows this rank sums
+      const int groups = r0 / 4;
+      const int t = tile0;
+      for (int u = et; u < groups * NT; u += 32 * NUM_EPI_WARPS) {
+        const int m = u / groups;
+        const int row = rank * r0 + 4 * (u % groups);
+        const int n = t * BMW + row;
+        if (m >= p.M || n >= p.N) continue;
+        const uint32_t off = static_cast<uint32_t>(m * BMW + row) * 4u;
+        float4 sum = ld_dsmem_f4(map_to_rank(s_part + off, 0));
+        for (int j = 1; j < split; ++j) {
+          const float4 v = ld_dsmem_f4(map_to_rank(s_part + off, j));
+          sum.x += v.x;
+          sum.y += v.y;
+          sum.z += v.z;
+          sum.w += v.w;
+        }
+        const float4 lr = ld_dsmem_f4(map_to_rank(s_lrt + off, rank));
+        const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+        const float lv[4] = {lr.x, lr.y, lr.z, lr.w};
+        uint32_t packed[2];
+#pragma unroll
+        for (int k = 0; k < 4; k += 2) {
+          float o[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float wc = __bfloat162float(p.wcscales[n + k + e]) * __bfloat162float(p.wtscale[0]);
+            const float bs = p.bias != nullptr ? __bfloat162float(p.bias[n + k + e]) : 0.f;
+            o[e] = fmaf(sv[k + e], wc, lv[k + e] + bs);
+          }
+          __nv_bfloat162 h = __floats2bfloat162_rn(o[0], o[1]);
+          packed[k / 2] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        st_global_v2(p.y + static_cast<size_t>(m) * p.ldy + n, packed[0], packed[1]);
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();
   }
 
   // ----------------------------------------------------------- teardown --

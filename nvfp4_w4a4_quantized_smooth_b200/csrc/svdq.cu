@@ -27,6 +27,8 @@ struct DeviceInfo {
   // Max co-resident clusters of the activation kernel, by (tile height
   // 64 / 128, split 1..8); -1 = not queried yet.
   int kq_clusters[2][svdq::kq::MAX_SPLIT + 1];
+  // Max co-resident clusters of the few-token GEMM by K split (1..8).
+  int ks_clusters[9];
 };
 
 std::mutex g_mu;
@@ -53,6 +55,7 @@ int device_setup(DeviceInfo** out) {
     d.num_sms = sms;
     for (auto& row : d.kq_clusters)
       for (int& v : row) v = -1;
+    for (int& v : d.ks_clusters) v = -1;
     if (d.sm100) {
       using namespace svdq;
       if (cudaFuncSetAttribute(kq::quantize_act_kernel<64, true, false>,
@@ -144,9 +147,51 @@ int launch_status() {
   return e == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
+// How many clusters of `split` few-token GEMM CTAs can be resident at once
+// on this device (cached).
+int ks_max_clusters(DeviceInfo* d, int split) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int& slot = d->ks_clusters[split];
+  if (slot >= 0) return slot;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(split * 256, 1, 1);
+  cfg.blockDim = dim3(svdq::ks::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = svdq::ks::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(
+          &n, reinterpret_cast<const void*>(svdq::ks::w4a4_linear_small_kernel<true>), &cfg) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  slot = n;
+  return n;
+}
+
+// K split of the few-token GEMM: the largest of 2, 4, 8 that keeps every
+// CTA on its own SM in one wave (all clusters co-resident) and gives each
+// CTA at least one K step of 256; else 1 (one CTA per tile, persistent).
+int ks_plan(DeviceInfo* d, int n_tiles, int num_k) {
+  int best = 1;
+  for (int split = 2; split <= 8; split *= 2) {
+    if (num_k < split || n_tiles * split > d->num_sms) break;
+    if (ks_max_clusters(d, split) < n_tiles) break;
+    best = split;
+  }
+  return best;
+}
+
 // The GEMM for M <= 64 tokens (ks_w4a4_linear_small.cuh): weights as the
-// 128-row MMA operand, one CTA per 128 weight rows.  Arguments as checked
-// by svdq_w4a4_linear.
+// 128-row MMA operand, one CTA per 128 weight rows and K range.  Arguments
+// as checked by svdq_w4a4_linear.
 int launch_small(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
                  const uint16_t* lowrank, const uint8_t* qweight, const void* wscales_tiled,
                  const uint16_t* wcscales, const uint16_t* wtscale, const uint16_t* proj_up,
@@ -181,22 +226,30 @@ int launch_small(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
   p.wcscales = reinterpret_cast<const __nv_bfloat16*>(wcscales);
   p.wtscale = reinterpret_cast<const __nv_bfloat16*>(wtscale);
   p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  p.y = reinterpret_cast<__nv_bfloat16*>(y);
   p.M = M;
   p.N = N;
   p.K = K;
+  p.ldy = ldy;
   p.n_tiles = (N + ks::BMW - 1) / ks::BMW;
-  const int grid = p.n_tiles < d->num_sms ? p.n_tiles : d->num_sms;
+  p.split = ks_plan(d, p.n_tiles, K / ks::BK);
+  const int grid =
+      p.split > 1 ? p.n_tiles * p.split : (p.n_tiles < d->num_sms ? p.n_tiles : d->num_sms);
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(ks::NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = ks::SMEM_BYTES;
   cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.split;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.split > 1 ? 2 : 1;
   const cudaError_t e =
       lr ? cudaLaunchKernelEx(&cfg, ks::w4a4_linear_small_kernel<true>, tm_w, tm_x, tm_sw, tm_p,
                               tm_l, tm_y, p)
