@@ -36,6 +36,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "SVDQ W4A4 linear TFLOP/s & % of dense NVFP4 roofline at DiT shapes"
+SMALL_M = 64          # svdq_w4a4_linear runs its few-token GEMM at M <= 64
 UNIT = "TFLOP/s"
 R = 128
 L2_BYTES = 126 * 1024 * 1024
@@ -319,6 +320,35 @@ def bench_ours(args, world, rank, local):
         for i in range(K_steps):
             run_step(svdq, sets[i % nsets], stream, evs[i])
         torch.cuda.synchronize(dev)
+        # The same steps from a CUDA graph (one step per rotating set,
+        # captured once, replayed): what the kernels take without the
+        # per-call host cost, which dominates at few tokens.  Reported
+        # beside the stream number.
+        graph = None
+        if not args.no_graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for j in range(nsets):
+                    run_step(svdq, sets[j], stream)
+            for _ in range(2):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            reps = max(1, -(-K_steps // nsets))
+            gs = torch.cuda.Event(enable_timing=True)
+            ge = torch.cuda.Event(enable_timing=True)
+            barrier(world)
+            gs.record(stream)
+            for _ in range(reps):
+                g.replay()
+            ge.record(stream)
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            gms = max_over_ranks(gs.elapsed_time(ge), world)
+            graph = {"value": round(job_value(one, reps * nsets, world, gms), 2), "unit": UNIT,
+                     "ms_per_step": round(gms / (reps * nsets), 5), "steps": reps * nsets,
+                     "what": f"one step per rotating set captured once in a CUDA graph, "
+                             f"replayed {reps} times"}
+            del g
         clocks.stop()
         svdq.check_device_error(stream)
 
@@ -342,8 +372,28 @@ def bench_ours(args, world, rank, local):
     t_roof_step = max(one / (fp4_peak * 1e12), (bytes_kq + bytes_kg) / (hbm * 1e9))
     step_s = elapsed_ms * 1e-3 / K_steps
     kg_tflops = flops_kg / (kg_avg * 1e-3) / 1e12
+    kg_gbs = bytes_kg / (kg_avg * 1e-3) / 1e9
     kq_gbs = bytes_kq / (kq_avg * 1e-3) / 1e9
-    traffic = load_traffic("w4a4_linear_kernel")
+    # M <= 64 runs the few-token GEMM, whose bytes (the weights) outweigh
+    # its flops at the measured peaks
+    kg_name = "w4a4_linear_small_kernel" if M <= SMALL_M else "w4a4_linear_kernel"
+    kg_hbm_bound = bytes_kg / (hbm * 1e9) > flops_kg / (fp4_peak * 1e12)
+    traffic = None if kg_name != "w4a4_linear_kernel" else load_traffic("w4a4_linear_kernel")
+    if kg_hbm_bound:
+        roofline = {"bound": "hbm", "kernel": kg_name, "achieved": round(kg_gbs, 1),
+                    "peak": round(hbm, 1), "unit": "GB/s", "frac": round(kg_gbs / hbm, 4),
+                    "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth",
+                    "algorithmic_bytes_per_launch": bytes_kg}
+    else:
+        roofline = {"bound": "tensor", "kernel": kg_name, "achieved": round(kg_tflops, 1),
+                    "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(kg_tflops / fp4_peak, 4), "traffic": traffic,
+                    "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal "
+                                   "FP4:BF16 dense ratio)",
+                    "algorithmic_flops_per_launch": flops_kg}
+    roofline.update({"avg_launch_ms": round(kg_avg, 5),
+                     "timing": "CUDA events around each launch on its stream, second pass "
+                               "of the timed steps"})
 
     # end to end through the public API with host buffers
     e2e = None if args.no_e2e else bench_e2e(args, svdq, sets[0], dev, M, K, N, world, r)
@@ -361,23 +411,16 @@ def bench_ours(args, world, rank, local):
                    "l2": f"inputs larger than L2: {nsets} rotating sets x "
                          f"{per_set / 2**20:.0f} MiB",
                    "repack_us": round(repack_us, 1),
-                   "roofline_frac_of_step": round(t_roof_step / step_s, 4)},
-        "roofline": {"bound": "tensor", "kernel": "w4a4_linear_kernel",
-                     "achieved": round(kg_tflops, 1), "peak": round(fp4_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(kg_tflops / fp4_peak, 4),
-                     "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal "
-                                    "FP4:BF16 dense ratio)",
-                     "algorithmic_flops_per_launch": flops_kg,
-                     "avg_launch_ms": round(kg_avg, 5),
-                     "timing": "CUDA events around each launch on its stream, second pass "
-                               "of the timed steps"},
+                   "roofline_frac_of_step": round(t_roof_step / step_s, 4),
+                   "cuda_graph": graph},
+        "roofline": roofline,
         "kernels": {
             "quantize_act_kernel": {"avg_ms": round(kq_avg, 5), "bytes": bytes_kq,
                                     "GB/s": round(kq_gbs, 1), "peak_GB/s": hbm,
                                     "frac": round(kq_gbs / hbm, 4), "bound": "hbm"},
-            "w4a4_linear_kernel": {"avg_ms": round(kg_avg, 5), "flops": flops_kg,
-                                   "TFLOP/s": round(kg_tflops, 1), "bytes": bytes_kg},
+            kg_name: {"avg_ms": round(kg_avg, 5), "flops": flops_kg,
+                      "TFLOP/s": round(kg_tflops, 1), "bytes": bytes_kg,
+                      "GB/s": round(kg_gbs, 1)},
         },
         "e2e": e2e,
         "gpu_launches": 2 * K_steps,
