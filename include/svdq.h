@@ -181,7 +181,8 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
 
 /* Launch shape svdq_quantize_act uses on the current device for an [M, K]
  * input with the low-rank branch (R = 128): rows per tile (*bm, 64 or 128) and the number of K ranges per
- * tile (*split: 1, 2, 4 or 8 CTAs of a cluster, at least 256 k each),
+ * tile (*split: 1, 2, 4, 8 or 16 CTAs of a cluster, at least 256 k each
+ * up to 8 and at least 128 k each with 16),
  * chosen to occupy the most SMs in one wave.  For inspection and tests;
  * needs a device. */
 int svdq_quantize_plan(int M, int K, int* bm, int* split);

@@ -83,7 +83,7 @@ constexpr int NUM_THREADS = 64 + NUM_QTHREADS;
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BUDGET = 227 * 1024;
 constexpr int PART_STRIDE = R + 4;     // floats per row of a staged partial (bank spread)
-constexpr int MAX_SPLIT = 8;
+constexpr int MAX_SPLIT = 16;
 
 // LR: the layer has the low-rank branch (R = 128); without it (R = 0, the
 // plain NVFP4 layer) a stage carries only x and smooth, there is no MMA,
@@ -526,20 +526,23 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
         const int m = u / (R / 4);
         const int c4 = u % (R / 4);
         const uint32_t off = s_ring + (m * PART_STRIDE + 4 * c4) * 4;
-        // All ranks' values are requested before the first add (the
+        // Eight ranks' values are requested before their first add (the
         // remote loads overlap); the sum still runs in rank order.
-        float4 t[MAX_SPLIT];
-#pragma unroll
-        for (int src = 0; src < MAX_SPLIT; ++src)
-          if (src < p.split) t[src] = ld_dsmem_f4(map_to_rank(off, static_cast<uint32_t>(src)));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int b0 = 0; b0 < p.split; b0 += 8) {
+          float4 t[8];
 #pragma unroll
-        for (int src = 0; src < MAX_SPLIT; ++src) {
-          if (src < p.split) {
-            acc.x += t[src].x;
-            acc.y += t[src].y;
-            acc.z += t[src].z;
-            acc.w += t[src].w;
+          for (int j = 0; j < 8; ++j)
+            if (b0 + j < p.split)
+              t[j] = ld_dsmem_f4(map_to_rank(off, static_cast<uint32_t>(b0 + j)));
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (b0 + j < p.split) {
+              acc.x += t[j].x;
+              acc.y += t[j].y;
+              acc.z += t[j].z;
+              acc.w += t[j].w;
+            }
           }
         }
         const int row = mb * BM + m;

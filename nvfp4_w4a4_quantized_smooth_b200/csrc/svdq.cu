@@ -93,6 +93,19 @@ int device_setup(DeviceInfo** out) {
                                ks::SMEM_BYTES) != cudaSuccess)
         return SVDQ_ERR_CUDA;
     }
+    if (d.sm100) {
+      // 16-CTA clusters of the activation kernel (non-portable size); if
+      // the device refuses, the occupancy query reports none and the plan
+      // keeps to 8.
+      using namespace svdq;
+      const void* fns[] = {reinterpret_cast<const void*>(kq::quantize_act_kernel<64, true, false>),
+                           reinterpret_cast<const void*>(kq::quantize_act_kernel<128, true, false>),
+                           reinterpret_cast<const void*>(kq::quantize_act_kernel<64, true, true>)};
+      for (const void* fn : fns)
+        if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess)
+          cudaGetLastError();
+    }
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -306,6 +319,13 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
 // tile height that pads M the least, then to the taller tile (less
 // proj_down traffic per row), then to the smaller split.
 // If none fits (very large M), 128-row tiles without a split.
+// A K split gives every CTA at least 256 k (4 chunks of 64) up to 8 ranks,
+// and at least one 128-k stage with 16 ranks (a non-portable cluster size,
+// used where few row tiles leave SMs idle).
+bool kq_split_ok(int split, int chunks) {
+  return split == 1 || (split <= 8 ? 4 * split <= chunks : 2 * split <= chunks);
+}
+
 void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out, bool tall_ok = true) {
   const int chunks = K / svdq::kq::BKE;
   int best_bm = tall_ok ? 128 : 64, best_split = 1, best_ctas = -1, best_pad = 0;
@@ -313,7 +333,7 @@ void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out, bool tall
     if (bm == 128 && !tall_ok) continue;
     const int m_tiles = (M + bm - 1) / bm;
     const int pad = m_tiles * bm - M;
-    for (int split = 1; split <= svdq::kq::MAX_SPLIT && (split == 1 || 4 * split <= chunks);
+    for (int split = 1; split <= svdq::kq::MAX_SPLIT && kq_split_ok(split, chunks);
          split *= 2) {
       const int ctas = m_tiles * split;
       if (ctas > d->num_sms) break;
@@ -338,7 +358,7 @@ void kq_plan_plain(DeviceInfo* d, int M, int K, int* bm_out, int* split_out) {
   for (int bm : {128, 64}) {
     const int m_tiles = (M + bm - 1) / bm;
     const int pad = m_tiles * bm - M;
-    for (int split = 1; split <= svdq::kq::MAX_SPLIT && (split == 1 || 4 * split <= chunks);
+    for (int split = 1; split <= svdq::kq::MAX_SPLIT && kq_split_ok(split, chunks);
          split *= 2) {
       const int ctas = m_tiles * split;
       if (ctas > d->num_sms) break;

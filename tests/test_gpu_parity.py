@@ -75,7 +75,8 @@ def test_quantize_act_bit_exact_and_lowrank(M, K):
 
 def test_quantize_plans_fit_one_wave():
     # 64- or 128-row tiles; a K split forms a cluster of 2, 4 or 8 CTAs with
-    # at least 256 k each; the grid runs in one wave when it can.
+    # at least 256 k each, or of 16 with at least 128 k each; the grid runs
+    # in one wave when it can.
     s = H.svdq()
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     for M in (1, 16, 64, 100, 256, 1024, 4352, 17408, 40000):
@@ -83,7 +84,8 @@ def test_quantize_plans_fit_one_wave():
             bm, split = s.quantize_plan(M, K)
             tiles = -(-M // bm)
             assert bm in (64, 128), (M, K, bm)
-            assert split in (1, 2, 4, 8) and (split == 1 or 256 * split <= K), (M, K, split)
+            assert split in (1, 2, 4, 8, 16), (M, K, split)
+            assert split == 1 or (256 if split <= 8 else 128) * split <= K, (M, K, split)
             if tiles * split > sms:
                 assert split == 1 and bm == 128, (M, K, bm, split)
             if M <= 64:
