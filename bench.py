@@ -254,6 +254,36 @@ def set_bytes(d):
     return sum(v.numel() * v.element_size() for v in d.values() if isinstance(v, torch.Tensor))
 
 
+def gemm_kernel_name(M):
+    """The GEMM kernel svdq_w4a4_linear runs for M tokens."""
+    return "w4a4_linear_small_kernel" if M <= SMALL_M else "w4a4_linear_kernel"
+
+
+def gemm_roofline(M, bytes_kg, flops_kg, kg_avg_ms, hbm_gbs, fp4_tflops, peak_src, traffic):
+    """Roofline object of the GEMM launch: bound by HBM when its algorithmic
+    bytes take longer than its flops at the measured peaks (the few-token
+    GEMM streaming the weights), else by the FP4 tensor pipe."""
+    kg_s = kg_avg_ms * 1e-3
+    if bytes_kg / (hbm_gbs * 1e9) > flops_kg / (fp4_tflops * 1e12):
+        achieved = bytes_kg / kg_s / 1e9
+        out = {"bound": "hbm", "kernel": gemm_kernel_name(M), "achieved": round(achieved, 1),
+               "peak": round(hbm_gbs, 1), "unit": "GB/s", "frac": round(achieved / hbm_gbs, 4),
+               "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth",
+               "algorithmic_bytes_per_launch": bytes_kg}
+    else:
+        achieved = flops_kg / kg_s / 1e12
+        out = {"bound": "tensor", "kernel": gemm_kernel_name(M), "achieved": round(achieved, 1),
+               "peak": round(fp4_tflops, 1), "unit": "TFLOP/s",
+               "frac": round(achieved / fp4_tflops, 4), "traffic": traffic,
+               "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal "
+                              "FP4:BF16 dense ratio)",
+               "algorithmic_flops_per_launch": flops_kg}
+    out.update({"avg_launch_ms": round(kg_avg_ms, 5),
+                "timing": "CUDA events around each launch on its stream, second pass "
+                          "of the timed steps"})
+    return out
+
+
 def run_step(svdq, d, stream, ev=None):
     if ev is not None:
         ev[0].record(stream)
@@ -374,26 +404,9 @@ def bench_ours(args, world, rank, local):
     kg_tflops = flops_kg / (kg_avg * 1e-3) / 1e12
     kg_gbs = bytes_kg / (kg_avg * 1e-3) / 1e9
     kq_gbs = bytes_kq / (kq_avg * 1e-3) / 1e9
-    # M <= 64 runs the few-token GEMM, whose bytes (the weights) outweigh
-    # its flops at the measured peaks
-    kg_name = "w4a4_linear_small_kernel" if M <= SMALL_M else "w4a4_linear_kernel"
-    kg_hbm_bound = bytes_kg / (hbm * 1e9) > flops_kg / (fp4_peak * 1e12)
+    kg_name = gemm_kernel_name(M)
     traffic = None if kg_name != "w4a4_linear_kernel" else load_traffic("w4a4_linear_kernel")
-    if kg_hbm_bound:
-        roofline = {"bound": "hbm", "kernel": kg_name, "achieved": round(kg_gbs, 1),
-                    "peak": round(hbm, 1), "unit": "GB/s", "frac": round(kg_gbs / hbm, 4),
-                    "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth",
-                    "algorithmic_bytes_per_launch": bytes_kg}
-    else:
-        roofline = {"bound": "tensor", "kernel": kg_name, "achieved": round(kg_tflops, 1),
-                    "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                    "frac": round(kg_tflops / fp4_peak, 4), "traffic": traffic,
-                    "peak_source": f"{peak_src} bf16 burst x {FP4_OVER_BF16:g} (nominal "
-                                   "FP4:BF16 dense ratio)",
-                    "algorithmic_flops_per_launch": flops_kg}
-    roofline.update({"avg_launch_ms": round(kg_avg, 5),
-                     "timing": "CUDA events around each launch on its stream, second pass "
-                               "of the timed steps"})
+    roofline = gemm_roofline(M, bytes_kg, flops_kg, kg_avg, hbm, fp4_peak, peak_src, traffic)
 
     # end to end through the public API with host buffers
     e2e = None if args.no_e2e else bench_e2e(args, svdq, sets[0], dev, M, K, N, world, r)
