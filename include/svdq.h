@@ -168,8 +168,10 @@ int svdq_silu_mul_quantize_act(const uint16_t* a, const uint16_t* b, int M, int 
  * Limits: R in {0, 128}, K % 256 == 0, N % 32 == 0 (else
  * SVDQ_ERR_UNSUPPORTED).
  * For M <= 64 the product is computed transposed (the weights as the
- * 128-row MMA operand, one CTA per 128 columns of y); the result is the
- * same sum, accumulated in fp32 in another order. */
+ * 128-row MMA operand, one CTA per 128 columns of y and, where such tiles
+ * are few, the K steps split over a thread-block cluster whose fp32
+ * partials are summed in a fixed rank order); the result is the same
+ * sum, accumulated in fp32 in another order, and repeats bit for bit. */
 int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
                      const uint16_t* lowrank, const uint8_t* qweight,
                      const void* wscales_tiled, const uint16_t* wcscales,
