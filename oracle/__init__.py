@@ -19,6 +19,9 @@ What it computes, and from which passage:
   (E2M1 elements with one e4m3 scale per 16 elements along K, R = 128).
 * The E2M1 bit layout (1 sign, 2 exponent, 1 mantissa bit) of the
   Z-Image NVFP4 blog, section "NVFP4 技术背景 / 什么是 NVFP4？".
+* The input of the w2 feed-forward linear, silu(w1 x) * (w3 x), for the
+  feed-forward linears w1, w2, w3 the same blog names in "Z-Image NVFP4
+  模型变体" (``silu_mul``; the gated form is the reading taken).
 
 Everything is decoded to float64 and multiplied with plain NumPy.  Each
 function is pinned by ``tests/test_oracle_pins.py`` against closed forms,
@@ -44,4 +47,6 @@ from .svdq_ref import (  # noqa: F401
     dequant_weight,
     w4a4_linear,
     svdq_linear_from_x,
+    plain_linear_from_x,
+    silu_mul,
 )

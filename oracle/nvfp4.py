@@ -52,16 +52,32 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+# bfloat16: 8 significant bits, exponent range of float32.  Smallest normal
+# 2^-126; subnormals are multiples of 2^-133; the largest finite value is
+# (2 - 2^-7) 2^127 and anything at or above (2 - 2^-8) 2^127 rounds to inf.
+_BF16_MIN_NORMAL = 2.0 ** -126
+_BF16_SUBNORMAL_QUANTUM = 2.0 ** -133
+_BF16_OVERFLOW = (2.0 - 2.0 ** -8) * 2.0 ** 127
+
+
 def f64_to_bf16_bits_rne(values) -> np.ndarray:
     """Round float64 values to bfloat16 (nearest, ties to even), raw bits.
 
-    Rounds straight from float64 (no float32 step, so no double rounding).
-    Covers zeros and the normal range of bfloat16, which is all the tests
-    use; subnormal results and overflow are not handled.
+    Rounds straight from float64 (no float32 step, so no double rounding),
+    as IEEE 754 rounds to a binary format with 8 significant bits and
+    float32's exponent range: normal results keep 8 significant bits,
+    results below 2^-126 are rounded to a multiple of the subnormal
+    quantum 2^-133 (gradual underflow), and magnitudes from the overflow
+    threshold (2 - 2^-8) 2^127 up give infinity.  The sign is kept, also
+    for results that round to zero.
     """
     v = np.asarray(values, dtype=np.float64)
     m, e = np.frexp(v)                      # v = m * 2^e, 0.5 <= |m| < 1
-    r = np.ldexp(np.rint(m * 256.0), e - 8)  # 8 significant bits, half-even
+    normal = np.ldexp(np.rint(m * 256.0), e - 8)  # 8 significant bits, half-even
+    sub = np.rint(v / _BF16_SUBNORMAL_QUANTUM) * _BF16_SUBNORMAL_QUANTUM
+    r = np.where(np.abs(v) < _BF16_MIN_NORMAL, sub, normal)
+    r = np.where(np.abs(v) >= _BF16_OVERFLOW, np.copysign(np.inf, v), r)
+    r = np.copysign(r, v)                   # a result that rounds to 0 keeps its sign
     out = r.astype(np.float32).view(np.uint32) >> np.uint32(16)
     return out.astype(np.uint16)
 

@@ -39,6 +39,7 @@ import numpy as np
 
 from .nvfp4 import (
     bf16_bits_to_f64,
+    f64_to_bf16_bits_rne,
     decode_e2m1,
     decode_e4m3,
     encode_e2m1_rne_sat,
@@ -129,6 +130,98 @@ def svdq_linear_from_x(x_bits, smooth_bits, proj_down_bits, qweight, wscales,
     y = w4a4_linear(qact, ascales, qweight, wscales, wcscales_bits,
                     wtscale_bits, proj_up_bits, bias_bits, L)
     return y, qact, ascales, L
+
+
+def _bf16_rounding_slack(v):
+    """Distance of each float64 value from the nearest bf16 rounding
+    boundary (a midpoint between neighbouring bf16 values), relative to |v|."""
+    v = np.abs(np.asarray(v, dtype=np.float64))
+    m, e = np.frexp(v)
+    quantum = np.where(v < 2.0 ** -126, 2.0 ** -133, np.ldexp(1.0, e - 8))
+    frac = v / quantum - np.floor(v / quantum)      # exact: v / quantum is a power-of-2 scaling
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return np.abs(frac - 0.5) * quantum / v
+
+
+def _round_fraction_to_bf16_bits(f, sign_negative):
+    """Exact rational magnitude |f| > 0 -> bf16 bits, nearest, ties to even."""
+    from fractions import Fraction
+    f = abs(f)
+    e = f.numerator.bit_length() - f.denominator.bit_length()
+    if Fraction(2) ** e > f:
+        e -= 1                                      # now 2^e <= f < 2^(e+1)
+    q = Fraction(2) ** (max(e, -126) - 7)           # bf16 spacing there
+    n, rem = divmod(f, q)
+    n = int(n)
+    if rem * 2 > q or (rem * 2 == q and n % 2 == 1):
+        n += 1
+    val = n * q
+    bits = 0x7F80 if val >= 2 ** 128 else int(
+        np.array(float(val), dtype=np.float32).view(np.uint32) >> 16)
+    return bits | (0x8000 if sign_negative else 0)
+
+
+def _silu_mul_exact_bits(a: float, b: float) -> int:
+    """bf16 bits of silu(a) * b from 400-digit decimal arithmetic, rounded
+    exactly.  400 digits hold every product of two bf16 values exactly (a
+    bf16 value is an integer below 2^8 times a power of two no smaller than
+    2^-133, whose decimal expansion has fewer than 140 digits).  The exact
+    product is not a bf16 midpoint for a, b != 0 (it is transcendental);
+    where the 400-digit value still lands on one (a > 0 with exp(-a) below
+    the working precision), the exact value lies just inside it in
+    magnitude, because silu(a) = a sigma(a) with sigma(a) < 1, so it rounds
+    toward zero there."""
+    import decimal
+    from fractions import Fraction
+    ctx = decimal.Context(prec=400, Emin=-10 ** 9, Emax=10 ** 9)
+    da, db = decimal.Decimal(a), decimal.Decimal(b)
+    d = ctx.multiply(ctx.divide(da, ctx.add(1, ctx.exp(ctx.minus(da)))), db)
+    f = Fraction(d)
+    if f == 0:
+        return 0x8000 if (np.signbit(a) != np.signbit(b)) else 0
+    bits = _round_fraction_to_bf16_bits(f, f < 0)
+    if a > 0:
+        # a tie at this precision: take the magnitude just below it
+        mag = abs(f)
+        lo = _round_fraction_to_bf16_bits(mag - mag * Fraction(1, 10 ** 500), f < 0)
+        hi = _round_fraction_to_bf16_bits(mag + mag * Fraction(1, 10 ** 500), f < 0)
+        if lo != hi:
+            bits = lo
+    return bits
+
+
+def silu_mul(a_bits, b_bits):
+    """h = bf16(silu(a) * b), silu(a) = a / (1 + exp(-a)): the input of the
+    w2 linear of a DiT feed-forward block.
+
+    The Z-Image NVFP4 blog, section "Z-Image NVFP4 模型变体", names the
+    feed-forward linears w1, w2 and w3; the reading taken for how they
+    combine is the gated form w2(silu(w1 x) * (w3 x)) those names denote,
+    with a = w1's bf16 output and b = w3's.  h is the exact product rounded
+    once to bf16 (nearest, ties to even, with gradual underflow and
+    overflow to inf).
+
+    Steps: evaluate silu(a) * b in float64 (relative error a few 2^-53)
+    and round it; where that value lies within 2^-44 (relative) of a bf16
+    rounding boundary, float64 cannot decide the rounding, and the product
+    is evaluated again with 400-digit decimal arithmetic and rounded
+    exactly (``_silu_mul_exact_bits``).  For a below about -709 exp(-a)
+    overflows float64 and a / inf is a signed zero, which is also what the
+    exact value (below 2^-1000 in magnitude) rounds to.  Inputs must be
+    finite.  Returns raw bf16 bits, same shape.
+    """
+    a = bf16_bits_to_f64(a_bits)
+    b = bf16_bits_to_f64(b_bits)
+    assert a.shape == b.shape
+    assert np.all(np.isfinite(a)) and np.all(np.isfinite(b))
+    with np.errstate(over="ignore"):
+        v = a / (1.0 + np.exp(-a)) * b
+    out = f64_to_bf16_bits_rne(v)
+    near = (v != 0) & (_bf16_rounding_slack(v) <= 2.0 ** -44)
+    for i in np.flatnonzero(near.reshape(-1)):
+        out.reshape(-1)[i] = _silu_mul_exact_bits(float(a.reshape(-1)[i]),
+                                                   float(b.reshape(-1)[i]))
+    return out
 
 
 BF16_ONE = 0x3F80

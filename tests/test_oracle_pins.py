@@ -494,3 +494,158 @@ def test_quantize_shapes_and_dtypes():
     assert qact.shape == (3, 24) and qact.dtype == np.uint8
     assert asc.shape == (3, 3) and asc.dtype == np.uint8
     assert np.all((asc & 0x80) == 0)        # amax/6 >= 0 -> sign bit clear
+
+
+# ------------------------------------------------ bf16 rounding extremes ---
+
+def test_bf16_rounding_of_subnormals_and_overflow_matches_torch():
+    # float32 inputs are exact in float64, so the oracle's single rounding
+    # must agree with torch's float32 -> bfloat16 conversion (nearest-even
+    # on the bit pattern) also for float32 subnormals, the smallest normals
+    # and values near the float32 maximum.
+    rng = np.random.default_rng(21)
+    sub = rng.integers(1, 1 << 23, 20000, dtype=np.uint32)                 # float32 subnormals
+    small = rng.integers(1 << 23, 3 << 23, 20000, dtype=np.uint32)         # binades 2^-126, 2^-125
+    big = rng.integers(0x7F000000, 0x7F800000, 20000, dtype=np.uint32)     # up to the float32 max
+    ties = (rng.integers(0, 1 << 15, 6000, dtype=np.uint32) << 16) | 0x8000  # exact bf16 midpoints
+    u = np.concatenate([sub, small, big, ties])
+    u = np.concatenate([u, u | np.uint32(0x80000000)])
+    v32 = u.view(np.float32)
+    v32 = v32[np.isfinite(v32)]
+    want = torch.from_numpy(v32.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = nv.f64_to_bf16_bits_rne(v32.astype(np.float64))
+    assert np.array_equal(got, want)
+    # overflow threshold (2 - 2^-8) 2^127 and signed zeros, by hand
+    thr = (2.0 - 2.0 ** -8) * 2.0 ** 127
+    assert nv.f64_to_bf16_bits_rne(thr) == 0x7F80
+    assert nv.f64_to_bf16_bits_rne(np.nextafter(thr, 0)) == 0x7F7F
+    assert nv.f64_to_bf16_bits_rne(-2.0 ** -135) == 0x8000
+    assert nv.f64_to_bf16_bits_rne(2.0 ** -134) == 0x0000                    # tie -> even (0)
+    assert nv.f64_to_bf16_bits_rne(3 * 2.0 ** -134) == 0x0002                # tie -> even (2)
+
+
+# --------------------------------------------------------- SiLU * mul ---
+
+def _bf16_table():
+    """Every non-negative finite bf16 value, indexed by its bit pattern."""
+    u = (np.arange(0, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    return [float(v) for v in u]
+
+
+def _silu_mul_bits_mp(a, b, mp, table):
+    """bf16 bits of silu(a) * b from 50-digit mpmath arithmetic, rounded by
+    searching the table of bf16 values (ties to the even bit pattern; at or
+    above the overflow threshold, inf).  Written independently of the
+    oracle.  For a > 0 the product is taken as P - c with P = a b exact and
+    c = P exp(-a) / (1 + exp(-a)), and the side of the nearest midpoint is
+    decided from (|P| - mid) - |c|, so that c is never lost to the working
+    precision (mpmath's exponent range is unbounded)."""
+    import bisect
+    a, b = mp.mpf(a), mp.mpf(b)
+    if a == 0 or b == 0:
+        neg = (mp.sign(a) < 0) != (mp.sign(b) < 0)
+        return None if (a == 0) else (0x8000 if neg else 0)
+    if a > 0:
+        P = a * b
+        c = P * mp.exp(-a) / (1 + mp.exp(-a))
+        x = P - c
+        above = lambda mid: (abs(P) - mid) - abs(c)           # sign of |x| - mid
+    else:
+        e = mp.exp(a)
+        x = a * e / (1 + e) * b
+        above = lambda mid: abs(x) - mid
+    sign = 0x8000 if x < 0 else 0
+    if above(mp.mpf((2.0 - 2.0 ** -8) * 2.0 ** 127)) >= 0:
+        return sign | 0x7F80
+    i = max(bisect.bisect_right(table, float(abs(x))) - 1, 0)
+    for _ in range(2):                       # float(|x|) may sit one entry low
+        if i + 1 < len(table):
+            d = above(mp.mpf(table[i]) / 2 + mp.mpf(table[i + 1]) / 2)
+            if d > 0 or (d == 0 and i % 2 == 1):
+                i += 1
+                continue
+        break
+    return sign | i
+
+
+def test_silu_mul_every_bf16_input_against_mpmath():
+    # silu(a) for every finite bf16 a (b = 1 and b = -0.75), against 50-digit
+    # mpmath arithmetic rounded by a table search.
+    mp = pytest.importorskip("mpmath").mp
+    mp.dps = 50
+    table = _bf16_table()
+    pos = np.arange(0, 0x7F80, dtype=np.uint16)
+    a_bits = np.concatenate([pos, pos | np.uint16(0x8000)])
+    a = nv.bf16_bits_to_f64(a_bits)
+    for bv in (1.0, -0.75):
+        b_bits = np.full(a_bits.shape, bf16_bits_of([bv])[0], dtype=np.uint16)
+        got = oracle.silu_mul(a_bits, b_bits)
+        want = np.array([_silu_mul_bits_mp(x, bv, mp, table)
+                         if x != 0 else (0x8000 if (np.signbit(x) != (bv < 0)) else 0)
+                         for x in a], dtype=np.uint16)
+        bad = np.flatnonzero(got != want)
+        assert bad.size == 0, (bv, [(a[i], hex(got[i]), hex(want[i])) for i in bad[:5]])
+
+
+def test_silu_mul_random_products_against_mpmath():
+    # Products spread over the whole bf16 range: outputs near the smallest
+    # normal and in the subnormal range, large negative a where exp(-a) is
+    # huge, and large outputs.
+    mp = pytest.importorskip("mpmath").mp
+    mp.dps = 50
+    table = _bf16_table()
+    rng = np.random.default_rng(22)
+    n = 6000
+    a = np.concatenate([rng.standard_normal(n) * 4, rng.uniform(-100, -80, n),
+                        rng.uniform(-30, 30, n), np.exp(rng.uniform(-20, 40, n))])
+    b = np.concatenate([rng.standard_normal(n), np.exp(rng.uniform(-60, 60, n)) * rng.choice([-1, 1], n),
+                        np.exp(rng.uniform(-90, -80, n)) * rng.choice([-1, 1], n),
+                        rng.standard_normal(n) * 1e-30])
+    a_bits = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    b_bits = torch.from_numpy(b).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    av, bv = nv.bf16_bits_to_f64(a_bits), nv.bf16_bits_to_f64(b_bits)
+    keep = np.isfinite(av) & np.isfinite(bv) & (av != 0) & (bv != 0)
+    a_bits, b_bits, av, bv = a_bits[keep], b_bits[keep], av[keep], bv[keep]
+    got = oracle.silu_mul(a_bits, b_bits)
+    want = np.array([_silu_mul_bits_mp(x, y, mp, table) for x, y in zip(av, bv)],
+                    dtype=np.uint16)
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, [(av[i], bv[i], hex(got[i]), hex(want[i])) for i in bad[:5]]
+    # the sample does reach the subnormal outputs and the region a < -87
+    assert np.any((got & 0x7F80) == 0) and np.any(av < -87)
+
+
+def test_silu_mul_closed_forms():
+    # silu(0) = 0 with the sign of the product; silu(a) * b for large a is
+    # a * b rounded, except where a * b is exactly a bf16 midpoint: silu(a)
+    # is then just below a, so the product rounds toward zero; for large
+    # negative a the product is a tiny value of the opposite sign to b.
+    z = bf16_bits_of([0.0, -0.0, 0.0, -0.0])
+    b = bf16_bits_of([1.0, 1.0, -2.0, -2.0])
+    assert list(oracle.silu_mul(z, b)) == [0x0000, 0x8000, 0x8000, 0x0000]
+    rng = np.random.default_rng(23)
+    a = bf16_bits_of([float(v) for v in rng.integers(64, 128, 200)])       # silu(a) = a (1 - 2^-92..)
+    bb = torch.from_numpy(rng.standard_normal(200)).to(torch.bfloat16)
+    b_bits = bb.view(torch.int16).numpy().view(np.uint16)
+    prod = nv.bf16_bits_to_f64(a) * nv.bf16_bits_to_f64(b_bits)          # exact (16 bits)
+    pbits = (torch.from_numpy(prod.astype(np.float32)).view(torch.int32).numpy()
+             .view(np.uint32))
+    is_tie = (pbits & 0xFFFF) == 0x8000
+    trunc = (pbits >> 16).astype(np.uint16)                                 # toward zero
+    rne = torch.from_numpy(prod.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.silu_mul(a, b_bits)
+    assert np.array_equal(got[~is_tie], rne[~is_tie])
+    # planted ties: a = 1.5 * 2^k, b = 1 + 2^-7: a * b has 9 significant bits
+    a_t = bf16_bits_of([48.0, 96.0, 192.0, 384.0, 1536.0, 3072.0])
+    b_t = bf16_bits_of([1.0 + 2.0 ** -7] * 6)
+    p = nv.bf16_bits_to_f64(a_t) * (1.0 + 2.0 ** -7)
+    pu = p.astype(np.float32).view(np.uint32)
+    assert np.all((pu & 0xFFFF) == 0x8000)
+    assert np.array_equal(oracle.silu_mul(a_t, b_t), (pu >> 16).astype(np.uint16))
+    assert np.array_equal(got[is_tie], trunc[is_tie])
+    # large negative a: -a e^a b, tiny and of the opposite sign to b
+    an = bf16_bits_of([-40.0, -60.0, -80.0])
+    bn = bf16_bits_of([3.0, -3.0, 3.0])
+    h = nv.bf16_bits_to_f64(oracle.silu_mul(an, bn))
+    want = np.array([-40 * math.exp(-40) * 3, 60 * math.exp(-60) * 3, -80 * math.exp(-80) * 3])
+    assert np.all(np.abs(h - want) <= 2.0 ** -8 * np.abs(want))
