@@ -37,6 +37,7 @@ if ROOT not in sys.path:
 
 METRIC = "SVDQ W4A4 linear TFLOP/s & % of dense NVFP4 roofline at DiT shapes"
 SMALL_M = 64          # svdq_w4a4_linear runs its few-token GEMM at M <= 64
+PAIR_M = 129          # ... and its CTA-pair GEMM at M >= 129
 UNIT = "TFLOP/s"
 R = 128
 L2_BYTES = 126 * 1024 * 1024
@@ -84,6 +85,7 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "w4a4_linear_kernel": "kg_w4a4_linear.cuh",
+    "w4a4_linear_pair_kernel": "kg2_w4a4_linear_pair.cuh",
     "quantize_act_kernel": "kq_quantize_act.cuh",
 }
 
@@ -236,9 +238,14 @@ def make_sets(M, K, N, nsets, seed, dev, plain=False):
         L = synth.make_layer(M, K, N, seed=seed + i)
         d = {k: (None if v is None else v.to(dev)) for k, v in vars(L).items()}
         torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0 = time.perf_counter()
+        e0.record()
         d["wscales_tiled"] = svdq.repack_weights(d["wscales"])
+        e1.record()
         d["repack_s"] = time.perf_counter() - t0
+        e1.synchronize()
+        d["repack_gpu_ms"] = e0.elapsed_time(e1)
         d["qact"] = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
         d["asc"] = torch.empty(svdq.ascales_tiled_bytes(M, K), dtype=torch.uint8, device=dev)
         d["lr"] = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
@@ -256,7 +263,9 @@ def set_bytes(d):
 
 def gemm_kernel_name(M):
     """The GEMM kernel svdq_w4a4_linear runs for M tokens."""
-    return "w4a4_linear_small_kernel" if M <= SMALL_M else "w4a4_linear_kernel"
+    if M <= SMALL_M:
+        return "w4a4_linear_small_kernel"
+    return "w4a4_linear_pair_kernel" if M >= PAIR_M else "w4a4_linear_kernel"
 
 
 def gemm_roofline(M, bytes_kg, flops_kg, kg_avg_ms, hbm_gbs, fp4_tflops, peak_src, traffic):
@@ -320,6 +329,7 @@ def bench_ours(args, world, rank, local):
     nsets = max(3, -(-3 * L2_BYTES // per_set))
     sets = probe + make_sets(M, K, N, nsets - 1, seed + 1, dev, plain)
     repack_us = 1e6 * statistics.median(d["repack_s"] for d in sets)
+    repack_gpu_us = 1e3 * statistics.median(d["repack_gpu_ms"] for d in sets)
 
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
@@ -405,7 +415,7 @@ def bench_ours(args, world, rank, local):
     kg_gbs = bytes_kg / (kg_avg * 1e-3) / 1e9
     kq_gbs = bytes_kq / (kq_avg * 1e-3) / 1e9
     kg_name = gemm_kernel_name(M)
-    traffic = None if kg_name != "w4a4_linear_kernel" else load_traffic("w4a4_linear_kernel")
+    traffic = load_traffic(kg_name) if kg_name in KERNEL_SOURCES else None
     roofline = gemm_roofline(M, bytes_kg, flops_kg, kg_avg, hbm, fp4_peak, peak_src, traffic)
 
     # end to end through the public API with host buffers
@@ -424,6 +434,11 @@ def bench_ours(args, world, rank, local):
                    "l2": f"inputs larger than L2: {nsets} rotating sets x "
                          f"{per_set / 2**20:.0f} MiB",
                    "repack_us": round(repack_us, 1),
+                   "repack_gpu_us": round(repack_gpu_us, 1),
+                   "repack_timing": ("repack_us: host wall time of svdq_repack_weights, which "
+                                     "synchronizes to read back the bad-scale count; "
+                                     "repack_gpu_us: CUDA events around the call on its "
+                                     "stream (counter reset, repack kernel, readback)"),
                    "roofline_frac_of_step": round(t_roof_step / step_s, 4),
                    "cuda_graph": graph},
         "roofline": roofline,

@@ -70,7 +70,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 7
+#define SVDQ_ABI_VERSION 8
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -101,7 +101,11 @@ size_t svdq_lowrank_bytes(int M, int R);
  *                  completely (padding rows get scale 0).
  * The GEMM reads scales as unsigned e4m3, so a byte with the sign bit set,
  * or a NaN code (0x7F), is rejected: the call then returns
- * SVDQ_ERR_INVALID_ARG.  To report that, this call SYNCHRONIZES `stream`. */
+ * SVDQ_ERR_INVALID_ARG.  To report that, this call SYNCHRONIZES `stream`.
+ * The bad bytes are counted in one device-wide word per device, so
+ * concurrent calls (from other host threads, on any stream) are
+ * serialized by a process-wide lock held from the counter's reset to its
+ * readback; each call reports only its own input. */
 int svdq_repack_weights(const uint8_t* wscales, int N, int K,
                         void* wscales_tiled, void* stream);
 
@@ -171,7 +175,11 @@ int svdq_silu_mul_quantize_act(const uint16_t* a, const uint16_t* b, int M, int 
  * 128-row MMA operand, one CTA per 128 columns of y and, where such tiles
  * are few, the K steps split over a thread-block cluster whose fp32
  * partials are summed in a fixed rank order); the result is the same
- * sum, accumulated in fp32 in another order, and repeats bit for bit. */
+ * sum, accumulated in fp32 in another order.  The split depends on the
+ * shape, the device's SM count and the clusters it can co-schedule
+ * (svdq_linear_plan), so results repeat bit for bit for the same shape on
+ * the same device with the same SMs available; across devices or SM
+ * counts they may differ in the last bits of the fp32 sums. */
 int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
                      const uint16_t* lowrank, const uint8_t* qweight,
                      const void* wscales_tiled, const uint16_t* wcscales,
@@ -185,9 +193,29 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
  * input with the low-rank branch (R = 128): rows per tile (*bm, 64 or 128) and the number of K ranges per
  * tile (*split: 1, 2, 4, 8 or 16 CTAs of a cluster, at least 256 k each
  * up to 8 and at least 128 k each with 16),
- * chosen to occupy the most SMs in one wave.  For inspection and tests;
- * needs a device. */
+ * chosen to occupy the most SMs in one wave.  The K ranges of a tile are
+ * [r * (K/64) / split, (r + 1) * (K/64) / split) in units of 64 k, so they
+ * differ by at most 64 k when K/64 is not a multiple of split.  The
+ * summation order of L (and so its last bits) depends on this plan, which
+ * depends on the device's SM count and cluster occupancy.  For inspection
+ * and tests; needs a device. */
 int svdq_quantize_plan(int M, int K, int* bm, int* split);
+
+/* Launch shape svdq_w4a4_linear uses on the current device for an
+ * M x N x K product (N % 32 == 0, K % 256 == 0): *kernel is
+ * SVDQ_GEMM_PAIRS (M > 128: persistent 256 x 256 output tiles, each on a
+ * pair of CTAs in a 2-CTA cluster sharing one tensor-core MMA, no K
+ * split), SVDQ_GEMM_TOKEN_MAJOR (64 < M <= 128: persistent 128 x 256 tiles
+ * on single CTAs) or SVDQ_GEMM_FEW_TOKENS (M <= 64: the transposed
+ * product, one 128-column tile of y per CTA and *split CTAs of a
+ * thread-block cluster per tile, each summing a range of
+ * [r * (K/256) / split, (r + 1) * (K/256) / split) K steps of 256); *grid
+ * is the number of CTAs launched.  For inspection and tests; needs a
+ * device. */
+#define SVDQ_GEMM_TOKEN_MAJOR 0
+#define SVDQ_GEMM_FEW_TOKENS 1
+#define SVDQ_GEMM_PAIRS 2
+int svdq_linear_plan(int M, int N, int K, int* kernel, int* split, int* grid);
 
 /* Inverse of the tile order, for tests and inspection: tiled scales of
  * `rows` rows -> out [rows, K/16] bytes, device.  `kind` says which order

@@ -130,25 +130,6 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   return v;
 }
 
-// Packed pairs of fp32 (lo in the low word) and their arithmetic.
-__device__ __forceinline__ uint64_t pk(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void upk(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
   asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
@@ -400,8 +381,11 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
               // swizzled places) for the MMA
               const uint4 b4 = lds_v4(s_y(s) + off);
               got ^= b4.x ^ b4.y ^ b4.z ^ b4.w;
-              v4 = make_uint4(silu_mul_bf16x2(v4.x, b4.x), silu_mul_bf16x2(v4.y, b4.y),
-                              silu_mul_bf16x2(v4.z, b4.z), silu_mul_bf16x2(v4.w, b4.w));
+              const uint32_t wa[4] = {v4.x, v4.y, v4.z, v4.w};
+              const uint32_t wb[4] = {b4.x, b4.y, b4.z, b4.w};
+              uint32_t wo[4];
+              silu_mul_words<4>(wa, wb, wo);
+              v4 = make_uint4(wo[0], wo[1], wo[2], wo[3]);
               st_shared_v4(s_x(s) + off, v4.x, v4.y, v4.z, v4.w);
             }
             xv[rr][4 * hh] = v4.x;

@@ -81,7 +81,8 @@ __global__ void unpack_scales_kernel(const uint8_t* __restrict__ tiled, int rows
   }
 }
 
-// out = silu(a) * b = a / (1 + exp(-a)) * b, fp32 math, bf16 result.
+// out = silu(a) * b = a / (1 + exp(-a)) * b rounded once to bf16
+// (silu_mul_words: fp32 with an fp64 path near bf16 rounding boundaries).
 __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
                                 const __nv_bfloat16* __restrict__ b,
                                 __nv_bfloat16* __restrict__ out, size_t n) {
@@ -95,8 +96,7 @@ __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
     const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w};
     const uint32_t wb[4] = {ub.x, ub.y, ub.z, ub.w};
     uint32_t wo[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) wo[j] = silu_mul_bf16x2(wa[j], wb[j]);
+    silu_mul_words<4>(wa, wb, wo);
     o4[i] = make_uint4(wo[0], wo[1], wo[2], wo[3]);
   }
   // tail
@@ -105,7 +105,7 @@ __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,
   if (tail0 + tid < n) {
     const float av = __bfloat162float(a[tail0 + tid]);
     const float bv = __bfloat162float(b[tail0 + tid]);
-    out[tail0 + tid] = __float2bfloat16_rn(silu_mul_f32(av, bv));
+    out[tail0 + tid] = __ushort_as_bfloat16(static_cast<unsigned short>(silu_mul_bf16_rn(av, bv)));
   }
 }
 

@@ -103,6 +103,18 @@ __device__ __forceinline__ bool svdq_wait(uint32_t bar, uint32_t parity, uint32_
   }
 }
 
+// Arrive on a barrier given by its shared::cluster address (this CTA's or
+// the peer CTA's of a CTA pair, from mapa).  Release at CTA scope, as for a
+// local barrier: the writes it publishes are tensor-memory stores ordered by
+// tcgen05.wait::st and tcgen05.fence::before_thread_sync before it, and a
+// cluster-scope release would fence all of this thread's memory operations
+// on every call.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(
+                   bar_cluster_addr)
+               : "memory");
+}
+
 // Bounded wait used on error paths only, to let copies already in flight
 // land before the block exits.  Never raises; gives up after `limit_ns`.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
@@ -113,22 +125,175 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-// ------------------------------------------------------------- SiLU * mul --
-// silu(a) * b = a / (1 + exp(-a)) * b in fp32 (the DiT feed-forward's gated
-// activation, w2's input), with CUDA's fast exponential and division
-// intrinsics (a few ulp of fp32, far below the bf16 rounding that follows).
-// One definition for every kernel that forms it, so that a fused and an
-// unfused path round to the same bf16.
-__device__ __forceinline__ float silu_mul_f32(float a, float b) {
-  return __fdividef(a, 1.0f + __expf(-a)) * b;
+// ------------------------------------------------- packed fp32 pairs --
+// Two fp32 values in one 64-bit register (lo in the low word) and the
+// paired arithmetic sm_100 issues as one instruction.
+__device__ __forceinline__ uint64_t pk(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
 }
-// Eight bf16 pairs (element 2i in the low half of word i) -> bf16 pairs of
-// silu(a) * b, nearest-even.
-__device__ __forceinline__ uint32_t silu_mul_bf16x2(uint32_t a, uint32_t b) {
-  const float lo = silu_mul_f32(__uint_as_float(a << 16), __uint_as_float(b << 16));
-  const float hi = silu_mul_f32(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u));
-  __nv_bfloat162 r = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&r);
+__device__ __forceinline__ void upk(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// ------------------------------------------------------------- SiLU * mul --
+// h = silu(a) * b = a / (1 + exp(-a)) * b rounded ONCE to bf16 (nearest,
+// ties to even, gradual underflow, overflow to inf): the input of the w2
+// linear of a DiT feed-forward block, w2(silu(w1 x) * (w3 x)).  One
+// definition for every kernel that forms it, so that a fused and an
+// unfused path give the same bits.
+//
+// Slow path, fp64 (never inlined): v = P sigma(a) with P = a b exact in
+// fp64 (two 8-bit significands) and sigma(a) = 1 / (1 + exp(-a)) for
+// a >= 0, exp(a) / (1 + exp(a)) below (no overflow), rounded to bf16
+// directly.  The exact product is never a bf16 midpoint for a, b != 0 (it
+// is transcendental), but the fp64 value can land on one, and then the
+// side is decided from the exact value's expansion:
+//   |a| < 2^-20: silu(a) b = P (1/2 + a/4 + O(a^3)), so the fp64 value is
+//                P / 2 = m and the exact one is beyond m iff a > 0;
+//   a > 0:       |v| = |P| - c with c = |P| exp(-a) / (1 + exp(-a)) > 0 and
+//                |P| - m exact, so it is beyond m iff |P| - m > c (for
+//                a > 37 the fp64 value is P itself and c decides);
+//   a < 0:       a coincidence of fp64 rounding; nearest-even is kept.
+__device__ __noinline__ uint32_t silu_mul_bf16_f64(float af, float bf) {
+  const double a = af, b = bf;
+  const double P = a * b;
+  const double t = exp(-fabs(a));
+  const double v = P * (a >= 0.0 ? 1.0 / (1.0 + t) : t / (1.0 + t));
+  const double av = fabs(v);
+  if (av == 0.0 || isinf(v)) return __bfloat16_as_ushort(__double2bfloat16(v));
+  // spacing of bf16 values at |v|: 2^(e - 7) for 2^e <= |v| (normal), 2^-133 below 2^-126
+  const int e = ilogb(av);
+  const double q = e < -126 ? 0x1p-133 : ldexp(1.0, e - 7);
+  const double x = av / q;   // a power-of-two scaling: exact
+  if (x - floor(x) != 0.5 || (a < 0.0 && fabs(a) >= 0x1p-20))
+    return __bfloat16_as_ushort(__double2bfloat16(v));
+  // v is exactly the midpoint m = |v| between floor(x) q and floor(x) q + q
+  const bool away = fabs(a) < 0x1p-20 ? a > 0.0 : (fabs(P) - av) > fabs(P) * (t / (1.0 + t));
+  const double r = (floor(x) + (away ? 1.0 : 0.0)) * q;
+  return __bfloat16_as_ushort(__double2bfloat16(v < 0.0 ? -r : r));
+}
+
+__device__ __forceinline__ float ex2_approx_ftz(float y) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx_ftz(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Fast path, fp32, one word of two elements (a, b: bf16 pairs, element 0
+// in the low half).  t = exp(-|a|) is 2^y with y = -|a| log2(e) split into
+// y_hi = fl(-|a| L) and the remainder y_lo (exact by FMA, plus
+// -|a| (log2 e - L)) -- the argument reduction of Cody and Waite ("Software
+// Manual for the Elementary Functions", 1980) -- so t = ex2(y_hi)
+// (1 + y_lo ln 2) with |y_lo| < 2^-16; then silu(a) b = a b / (1 + t) for
+// a >= 0 and (a t) b / (1 + t) below, with the reciprocal of 1 + t in
+// [1, 2].  With ex2.approx and rcp.approx within 2^-21 and 2^-22
+// (relative) and the float roundings, the result is within 2^-20 of the
+// exact product, under 16 float ulps, so its nearest-even rounding to bf16
+// is that of the exact value unless the float lies within 64 ulps of a bf16
+// midpoint (low 16 bits within 64 of 0x8000).  Inputs outside the range of
+// that bound show up in the result and are sent to the fp64 path too: for
+// |a| > 87 t flushes to zero, which for a < 0 gives a zero product and for
+// a > 0 the product a b itself (exact; only a midpoint, caught by the
+// window, can round differently from the exact value just inside it); a
+// zero, subnormal or infinite bf16 result (zeros, subnormal operands,
+// overflow of a b) is sent over as well.  Returns the bf16 pair; bits 0 and
+// 1 of `slow` flag the elements the fp64 path must decide.
+__device__ __forceinline__ uint32_t silu_mul_fast2(uint32_t a, uint32_t b, uint32_t& slow) {
+  const uint64_t kNegL = pk(-1.44269502f, -1.44269502f);     // -log2(e) rounded to float
+  const uint64_t kL = pk(1.44269502f, 1.44269502f);
+  const uint64_t kLlo = pk(1.92596299e-08f, 1.92596299e-08f); // log2(e) - 1.44269502f
+  const uint64_t kNegLn2 = pk(-0.693147182f, -0.693147182f);
+  const uint64_t kOne = pk(1.0f, 1.0f);
+  const uint64_t av = pk(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+  const uint64_t bv = pk(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u));
+  const uint64_t abs_a = pk(__uint_as_float((a << 17) >> 1), __uint_as_float((a & 0x7FFF0000u)));
+  const uint64_t yhi = mul2(abs_a, kNegL);                    // fl(-|a| L)
+  const uint64_t r1 = fma2(abs_a, kL, yhi);                   // |a| L + y_hi, exact
+  const uint64_t r2 = fma2(abs_a, kLlo, r1);                  // -y_lo
+  const uint64_t corr = fma2(r2, kNegLn2, kOne);              // 1 + y_lo ln 2
+  float y0, y1;
+  upk(yhi, y0, y1);
+  const uint64_t t = mul2(pk(ex2_approx_ftz(y0), ex2_approx_ftz(y1)), corr);
+  float d0, d1;
+  upk(add2(t, kOne), d0, d1);
+  const uint64_t rcp = pk(rcp_approx_ftz(d0), rcp_approx_ftz(d1));
+  const uint64_t P = mul2(av, bv);                            // a b, exact
+  const uint64_t Q = mul2(mul2(av, t), bv);                   // (a t) b
+  float p0, p1, q0, q1;
+  upk(P, p0, p1);
+  upk(Q, q0, q1);
+  const uint64_t num = pk((a & 0x8000u) ? q0 : p0, (a & 0x80000000u) ? q1 : p1);
+  float v0, v1;
+  upk(mul2(num, rcp), v0, v1);
+  uint32_t h;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(v1), "f"(v0));
+  const uint32_t u0 = __float_as_uint(v0), u1 = __float_as_uint(v1);
+  // result exponent field 0 (zero, subnormal) or 0xFF (inf) in either half
+  const uint32_t e = h & 0x7F807F80u;
+  const uint32_t zero_sub = ~((e | 0x80008000u) - 0x00800080u) & 0x80008000u;
+  const uint32_t inf = (e + 0x00800080u) & 0x80008000u;
+  const uint32_t bad = zero_sub | inf;
+  slow = (((u0 & 0xFFFFu) - 0x7FC0u) <= 0x80u || (bad & 0x8000u) ? 1u : 0u) |
+         (((u1 & 0xFFFFu) - 0x7FC0u) <= 0x80u || (bad & 0x80000000u) ? 2u : 0u);
+  return h;
+}
+
+// One element, either path.
+__device__ __forceinline__ uint32_t silu_mul_bf16_rn(float a, float b) {
+  uint32_t slow;
+  const uint32_t h = silu_mul_fast2(__float_as_uint(a) >> 16, __float_as_uint(b) >> 16, slow);
+  return (slow & 1u) ? silu_mul_bf16_f64(a, b) : (h & 0xFFFFu);
+}
+
+// NW words of bf16 pairs (element 0 in the low half): out = silu(a) * b,
+// bf16 pairs.  The fast path runs on every element first; the few it cannot
+// decide (about one in 500) are redone on the fp64 path afterwards, outside
+// the main loop, so that the common path stays a straight line of float
+// arithmetic.
+template <int NW>
+__device__ __forceinline__ void silu_mul_words(const uint32_t (&a)[NW], const uint32_t (&b)[NW],
+                                               uint32_t (&out)[NW]) {
+  uint32_t need = 0;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) {
+    uint32_t sl;
+    out[i] = silu_mul_fast2(a[i], b[i], sl);
+    need |= sl << (2 * i);
+  }
+  if (need != 0u) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) {
+      if (need & (1u << (2 * i)))
+        out[i] = (out[i] & 0xFFFF0000u) |
+                 silu_mul_bf16_f64(__uint_as_float(a[i] << 16), __uint_as_float(b[i] << 16));
+      if (need & (2u << (2 * i)))
+        out[i] = (out[i] & 0xFFFFu) | (silu_mul_bf16_f64(__uint_as_float(a[i] & 0xFFFF0000u),
+                                                         __uint_as_float(b[i] & 0xFFFF0000u))
+                                       << 16);
+    }
+  }
 }
 
 // ------------------------------------------------- dependent launches --
@@ -168,6 +333,19 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int3
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// 2-D tiled bulk tensor load into this CTA's shared memory whose completion
+// is signalled on a barrier of either CTA of the CTA pair (`bar` a
+// shared::cluster address): the operand loads of a cta_group::2 MMA.  No
+// multicast: each CTA loads its own half from this GPU's memory.
+__device__ __forceinline__ void tma_load_2d_cg2(uint32_t dst, const void* tmap, int32_t x,
+                                                int32_t y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::"
+      "bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
 
@@ -274,6 +452,60 @@ __device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
       "p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// ---- CTA pairs (cta_group::2): one MMA over both CTAs' operands ----------
+// TMEM allocation / release for the pair: one warp of EACH CTA executes it;
+// both CTAs get the same column range.
+__device__ __forceinline__ void tmem_alloc_cg2(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_cg2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_cg2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// Arrive on the barrier at this offset in every CTA of `cta_mask` once all
+// pair MMAs this thread issued so far have completed.
+__device__ __forceinline__ void tc_commit_cg2_mc(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+// Same, arriving on one barrier of this CTA.
+__device__ __forceinline__ void tc_commit_cg2(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+// Pair MMA, issued by the even CTA: M = 256 rows, rows [0, 128) from this
+// CTA's A and into its TMEM, [128, 256) from the odd CTA's; each CTA holds
+// half of B's N rows.  Descriptors and TMEM addresses are the same in both.
+__device__ __forceinline__ void mma_nvfp4_cg2(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t sfa_tmem,
+                                              uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f16_cg2(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

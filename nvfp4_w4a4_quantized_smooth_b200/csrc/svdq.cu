@@ -13,6 +13,7 @@
 #include "sm100_ptx.cuh"
 #include "kq_quantize_act.cuh"
 #include "kg_w4a4_linear.cuh"
+#include "kg2_w4a4_linear_pair.cuh"
 #include "ks_w4a4_linear_small.cuh"
 #include "kr_scales.cuh"
 
@@ -29,9 +30,15 @@ struct DeviceInfo {
   int kq_clusters[2][svdq::kq::MAX_SPLIT + 1];
   // Max co-resident clusters of the few-token GEMM by K split (1..8).
   int ks_clusters[9];
+  // Max co-resident CTA pairs of the pair GEMM; -1 = not queried yet.
+  int kg2_pairs = -1;
 };
 
 std::mutex g_mu;
+// Held by svdq_repack_weights across its reset / kernel / readback of the
+// device-wide bad-scale counter, so that concurrent repacks (other host
+// threads, other streams) cannot reset or read each other's count.
+std::mutex g_repack_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -90,7 +97,13 @@ int device_setup(DeviceInfo** out) {
                                ks::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(ks::w4a4_linear_small_kernel<false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ks::SMEM_BYTES) != cudaSuccess)
+                               ks::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kg2::w4a4_linear_pair_kernel<true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kg2::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kg2::w4a4_linear_pair_kernel<false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kg2::SMEM_BYTES) != cudaSuccess)
         return SVDQ_ERR_CUDA;
     }
     if (d.sm100) {
@@ -202,6 +215,61 @@ int ks_plan(DeviceInfo* d, int n_tiles, int num_k) {
   return best;
 }
 
+// Launch shape of the few-token GEMM for N output channels and K: the K
+// split (cluster size) and the grid.  svdq_linear_plan reports the same.
+void ks_shape(DeviceInfo* d, int N, int K, int* split, int* grid) {
+  const int n_tiles = (N + svdq::ks::BMW - 1) / svdq::ks::BMW;
+  *split = ks_plan(d, n_tiles, K / svdq::ks::BK);
+  *grid = *split > 1 ? n_tiles * *split : (n_tiles < d->num_sms ? n_tiles : d->num_sms);
+}
+
+// Grid of the token-major GEMM: one persistent CTA per SM, or one per tile
+// when tiles are fewer.
+int kg_grid(DeviceInfo* d, int M, int N) {
+  const int tiles = ((M + svdq::kg::BM - 1) / svdq::kg::BM) * ((N + svdq::kg::BN - 1) / svdq::kg::BN);
+  return tiles < d->num_sms ? tiles : d->num_sms;
+}
+
+// The token-major GEMM runs on CTA pairs (256 x 256 tiles) above this many
+// tokens; between the few-token limit and it, on single SMs (128 x 256).
+constexpr int kPairMinM = 129;
+
+// How many CTA pairs of the pair GEMM can be resident at once (cached).
+int kg2_max_pairs(DeviceInfo* d) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (d->kg2_pairs >= 0) return d->kg2_pairs;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * 256, 1, 1);
+  cfg.blockDim = dim3(svdq::kg2::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = svdq::kg2::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(
+          &n, reinterpret_cast<const void*>(svdq::kg2::w4a4_linear_pair_kernel<true>), &cfg) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  d->kg2_pairs = n;
+  return n;
+}
+
+// Grid of the pair GEMM (CTAs, two per pair): one persistent pair per two
+// SMs that the device co-schedules, or one per tile when tiles are fewer.
+int kg2_grid(DeviceInfo* d, int M, int N) {
+  const int tiles = ((M + svdq::kg2::BM - 1) / svdq::kg2::BM) * ((N + svdq::kg2::BN - 1) / svdq::kg2::BN);
+  int pairs = kg2_max_pairs(d);
+  if (pairs < 1) pairs = 1;
+  return 2 * (tiles < pairs ? tiles : pairs);
+}
+
 // The GEMM for M <= 64 tokens (ks_w4a4_linear_small.cuh): weights as the
 // 128-row MMA operand, one CTA per 128 weight rows and K range.  Arguments
 // as checked by svdq_w4a4_linear.
@@ -245,9 +313,8 @@ int launch_small(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
   p.K = K;
   p.ldy = ldy;
   p.n_tiles = (N + ks::BMW - 1) / ks::BMW;
-  p.split = ks_plan(d, p.n_tiles, K / ks::BK);
-  const int grid =
-      p.split > 1 ? p.n_tiles * p.split : (p.n_tiles < d->num_sms ? p.n_tiles : d->num_sms);
+  int grid = 0;
+  ks_shape(d, N, K, &p.split, &grid);
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(grid, 1, 1);
@@ -268,6 +335,69 @@ int launch_small(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
                               tm_l, tm_y, p)
          : cudaLaunchKernelEx(&cfg, ks::w4a4_linear_small_kernel<false>, tm_w, tm_x, tm_sw, tm_p,
                               tm_l, tm_y, p);
+  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
+  return launch_status();
+}
+
+// The token-major GEMM on CTA pairs (kg2_w4a4_linear_pair.cuh), 256 x 256
+// tiles.  Arguments as checked by svdq_w4a4_linear.
+int launch_pair(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
+                const uint16_t* lowrank, const uint8_t* qweight, const void* wscales_tiled,
+                const uint16_t* wcscales, const uint16_t* wtscale, const uint16_t* proj_up,
+                const uint16_t* bias, int M, int N, int K, int R, uint16_t* y, int ldy,
+                void* stream) {
+  namespace kg2 = svdq::kg2;
+  const bool lr = R != 0;
+  const uint64_t kb = static_cast<uint64_t>(K) / 2;
+  CUtensorMap tm_a, tm_b, tm_l, tm_p, tm_y;
+  if (make_tmap(&tm_a, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, kg2::BK_BYTES,
+                kg2::BM_CTA) ||
+      make_tmap(&tm_b, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, N, kb, kg2::BK_BYTES,
+                kg2::BN_CTA) ||
+      make_tmap(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(ldy) * 2,
+                kg2::OUT_COLS, 32))
+    return SVDQ_ERR_CUDA;
+  if (!lr) {
+    tm_l = tm_a;   // not read
+    tm_p = tm_b;
+  } else if (make_tmap(&tm_l, lowrank, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, M,
+                       static_cast<uint64_t>(R) * 2, 64, kg2::BM_CTA) ||
+             make_tmap(&tm_p, proj_up, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, R, N,
+                       static_cast<uint64_t>(R) * 2, 64, kg2::BN_CTA)) {
+    return SVDQ_ERR_CUDA;
+  }
+  kg2::Params p;
+  p.ascales_tiled = static_cast<const uint8_t*>(ascales_tiled);
+  p.wscales_tiled = static_cast<const uint8_t*>(wscales_tiled);
+  p.wcscales = reinterpret_cast<const __nv_bfloat16*>(wcscales);
+  p.wtscale = reinterpret_cast<const __nv_bfloat16*>(wtscale);
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.m_tiles = (M + kg2::BM - 1) / kg2::BM;
+  p.n_tiles = (N + kg2::BN - 1) / kg2::BN;
+  p.a_row_tiles = (M + 127) / 128;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(kg2_grid(d, M, N), 1, 1);
+  cfg.blockDim = dim3(kg2::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = kg2::SMEM_BYTES;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e =
+      lr ? cudaLaunchKernelEx(&cfg, kg2::w4a4_linear_pair_kernel<true>, tm_a, tm_b, tm_l, tm_p,
+                              tm_y, p)
+         : cudaLaunchKernelEx(&cfg, kg2::w4a4_linear_pair_kernel<false>, tm_a, tm_b, tm_l, tm_p,
+                              tm_y, p);
   if (e != cudaSuccess) return SVDQ_ERR_CUDA;
   return launch_status();
 }
@@ -434,6 +564,8 @@ int svdq_repack_weights(const uint8_t* wscales, int N, int K, void* wscales_tile
   const int rows_pad = (N + 255) / 256 * 256;
   const size_t words = static_cast<size_t>(rows_pad) * (K / 64);
   uint32_t zero = 0, bad = 0;
+  // One repack at a time per process: the counter is shared by every call.
+  std::lock_guard<std::mutex> lock(g_repack_mu);
   if (cudaMemcpyToSymbolAsync(svdq::kr::g_bad_scales, &zero, sizeof(zero), 0,
                               cudaMemcpyHostToDevice, s) != cudaSuccess)
     return SVDQ_ERR_CUDA;
@@ -592,6 +724,9 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   if (M <= svdq::ks::NT)
     return launch_small(d, qact, ascales_tiled, lowrank, qweight, wscales_tiled, wcscales,
                         wtscale, proj_up, bias, M, N, K, R, y, ldy, stream);
+  if (M >= kPairMinM)
+    return launch_pair(d, qact, ascales_tiled, lowrank, qweight, wscales_tiled, wcscales,
+                       wtscale, proj_up, bias, M, N, K, R, y, ldy, stream);
   CUtensorMap tm_a, tm_b, tm_l, tm_p, tm_y;
   if (make_tmap(&tm_a, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, svdq::kg::BK_BYTES,
                 svdq::kg::BM) ||
@@ -621,8 +756,7 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   p.K = K;
   p.m_tiles = (M + svdq::kg::BM - 1) / svdq::kg::BM;
   p.n_tiles = (N + svdq::kg::BN - 1) / svdq::kg::BN;
-  const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < d->num_sms ? tiles : d->num_sms;
+  const int grid = kg_grid(d, M, N);
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(grid, 1, 1);
@@ -641,6 +775,27 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
                               tm_y, p);
   if (e != cudaSuccess) return SVDQ_ERR_CUDA;
   return launch_status();
+}
+
+int svdq_linear_plan(int M, int N, int K, int* kernel, int* split, int* grid) {
+  if (!kernel || !split || !grid) return SVDQ_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 16 || K % 16) return SVDQ_ERR_SHAPE;
+  if (K % svdq::kg::BK || N % 32) return SVDQ_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  if (M <= svdq::ks::NT) {
+    *kernel = SVDQ_GEMM_FEW_TOKENS;
+    ks_shape(d, N, K, split, grid);
+  } else if (M >= kPairMinM) {
+    *kernel = SVDQ_GEMM_PAIRS;
+    *split = 1;
+    *grid = kg2_grid(d, M, N);
+  } else {
+    *kernel = SVDQ_GEMM_TOKEN_MAJOR;
+    *split = 1;
+    *grid = kg_grid(d, M, N);
+  }
+  return SVDQ_OK;
 }
 
 int svdq_quantize_plan(int M, int K, int* bm, int* split) {

@@ -29,9 +29,12 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 7
+ABI_VERSION = 8
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
+GEMM_TOKEN_MAJOR = 0
+GEMM_FEW_TOKENS = 1
+GEMM_PAIRS = 2
 
 # Every symbol include/svdq.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -48,6 +51,8 @@ SIGNATURES = {
     "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
     "svdq_silu_mul_quantize_act": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
     "svdq_quantize_plan": (_I, [_I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "svdq_linear_plan": (_I, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                              ctypes.POINTER(_I)]),
     "svdq_unpack_scales": (_I, [_P, _I, _I, _I, _P, _P]),
     "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
     "svdq_check_device_error": (_I, [_P]),
@@ -241,6 +246,16 @@ def quantize_plan(M: int, K: int):
     _check(_lib.svdq_quantize_plan(M, K, ctypes.byref(bm), ctypes.byref(split)),
            "svdq_quantize_plan")
     return bm.value, split.value
+
+
+def linear_plan(M: int, N: int, K: int):
+    """(kernel, K split, grid) svdq_w4a4_linear uses for M x N x K on this
+    device; kernel is GEMM_PAIRS, GEMM_TOKEN_MAJOR or GEMM_FEW_TOKENS."""
+    kernel, split, grid = _I(), _I(), _I()
+    _check(_lib.svdq_linear_plan(M, N, K, ctypes.byref(kernel), ctypes.byref(split),
+                                 ctypes.byref(grid)),
+           "svdq_linear_plan")
+    return kernel.value, split.value, grid.value
 
 
 def unpack_scales(scales_tiled: torch.Tensor, rows: int, K: int, kind: str = "act",

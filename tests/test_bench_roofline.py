@@ -17,7 +17,9 @@ def test_kernel_by_token_count():
     assert bench.gemm_kernel_name(1) == "w4a4_linear_small_kernel"
     assert bench.gemm_kernel_name(64) == "w4a4_linear_small_kernel"
     assert bench.gemm_kernel_name(65) == "w4a4_linear_kernel"
-    assert bench.gemm_kernel_name(4352) == "w4a4_linear_kernel"
+    assert bench.gemm_kernel_name(128) == "w4a4_linear_kernel"
+    assert bench.gemm_kernel_name(129) == "w4a4_linear_pair_kernel"
+    assert bench.gemm_kernel_name(4352) == "w4a4_linear_pair_kernel"
 
 
 def test_few_tokens_are_hbm_bound():
@@ -36,7 +38,7 @@ def test_dit_shape_is_tensor_bound():
     r = bench.gemm_roofline(4352, 138662914, 397871677440, 0.121, HBM, FP4, "measured",
                             90749184.0)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
-    assert r["kernel"] == "w4a4_linear_kernel"
+    assert r["kernel"] == "w4a4_linear_pair_kernel"
     assert abs(r["achieved"] - 397871677440 / 121e-6 / 1e12) < 0.1
     assert abs(r["frac"] - r["achieved"] / FP4) < 1e-4
     assert r["traffic"] == 90749184.0

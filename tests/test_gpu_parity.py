@@ -223,10 +223,9 @@ def test_plain_nvfp4_layer_full_size_qkv():
     M, K, N = synth.WORKLOADS[name]
     L = synth.make_layer(M, K, N, seed=synth.workload_seed(name))
     r = H.gpu_plain_layer(L, False)
-    rows = H.sample_rows(M, 32, seed=5)
-    y_ref, q_ref, a_ref = H.oracle_plain_y(L, False, rows=rows)
-    H.assert_quant_exact(r["qact"][rows], r["ascales"][rows], q_ref, a_ref, "plain qkv quant")
-    H.assert_y_close(r["y"][rows], y_ref, "plain qkv")
+    y_ref, q_ref, a_ref = H.oracle_plain_y(L, False)
+    H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, "plain qkv quant")
+    H.assert_y_close(r["y"], y_ref, "plain qkv")
 
 
 def test_linear_without_bias():
@@ -311,24 +310,21 @@ def test_output_row_stride():
 
 # ------------------------------------------------- full-size workloads ---
 
-def _full_size_check(name, n_rows=48):
+def _full_size_check(name):
+    """Every code, scale, L value and output of the workload against the
+    oracle (the fp64 product of the decoded operands)."""
     M, K, N = synth.WORKLOADS[name]
     L = synth.make_layer(M, K, N, seed=synth.workload_seed(name))
     r = H.gpu_layer(L)
-    if M * K <= 20_000_000:
-        # every code and scale of the whole activation
-        q_ref, a_ref = H.oracle_quant(L.x, L.smooth)
-        H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, name)
-    rows = H.sample_rows(M, n_rows, seed=M)
-    y_ref, q_ref, a_ref, L_ref = H.oracle_y(L, rows=rows)
-    H.assert_quant_exact(r["qact"][rows], r["ascales"][rows], q_ref, a_ref, name)
-    H.assert_y_close(r["y"][rows], y_ref, name)
-    H.assert_lowrank_close(r["lowrank"][rows], L_ref, name)
+    y_ref, q_ref, a_ref, L_ref = H.oracle_y(L)
+    H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, name)
+    H.assert_y_close(r["y"], y_ref, name)
+    H.assert_lowrank_close(r["lowrank"], L_ref, name)
     return L, r
 
 
 def test_full_size_layer_m128():
-    _full_size_check("layer_m128_k512_n512", n_rows=128)
+    _full_size_check("layer_m128_k512_n512")
 
 
 def test_full_size_qkv():
@@ -337,67 +333,71 @@ def test_full_size_qkv():
 
 @pytest.mark.parametrize("M", synth.OUT_PROJ_SWEEP_M)
 def test_full_size_out_proj_sweep(M):
-    _full_size_check(f"out_m{M}_k3840_n3840", n_rows=32)
+    _full_size_check(f"out_m{M}_k3840_n3840")
 
 
 def test_full_size_ffn_chain():
     # w1, w3 on the block input, h = silu(y1) * y3 from the GPU's own bf16
-    # outputs, then w2 on h; the oracle for w2 takes that h as its input.
+    # outputs (bit for bit the oracle's silu_mul of those outputs), then w2
+    # on h; the oracle for w2 takes that h as its input.
     s = H.svdq()
-    L1, r1 = _full_size_check("ffn_w1_m4352_k3840_n10240", n_rows=24)
+    L1, r1 = _full_size_check("ffn_w1_m4352_k3840_n10240")
     L3 = synth.make_layer(*synth.WORKLOADS["ffn_w3_m4352_k3840_n10240"],
                           seed=synth.workload_seed("ffn_w3_m4352_k3840_n10240"))
     L3.x = L1.x
     r3 = H.gpu_layer(L3)
+    y3_ref, *_ = H.oracle_y(L3)
+    H.assert_y_close(r3["y"], y3_ref, "w3")
     h = s.silu_mul(r1["y"].cuda(), r3["y"].cuda())
     s.check_device_error()
-    a = r1["y"].float()
-    want_h = (a * torch.sigmoid(a) * r3["y"].float()).to(torch.bfloat16)
     hd = h.cpu()
-    diff = (hd.float() - want_h.float()).abs()
-    assert (diff <= 2 ** -7 * want_h.float().abs() + 1e-6).all()
+    h_ref = oracle.silu_mul(H.bits(r1["y"]), H.bits(r3["y"]))
+    assert np.array_equal(H.bits(hd), h_ref), "silu(y1) * y3 differs from the oracle"
     L2 = synth.make_layer(*synth.WORKLOADS["ffn_w2_m4352_k10240_n3840"],
                           seed=synth.workload_seed("ffn_w2_m4352_k10240_n3840"))
     r2 = H.gpu_layer(L2, x_override=h)
-    rows = H.sample_rows(L2.M, 24, seed=2)
-    y_ref, q_ref, a_ref, _ = H.oracle_y(L2, rows=rows, x=hd)
-    H.assert_quant_exact(r2["qact"][rows], r2["ascales"][rows], q_ref, a_ref, "w2 quant")
-    H.assert_y_close(r2["y"][rows], y_ref, "w2")
+    y_ref, q_ref, a_ref, L_ref = H.oracle_y(L2, x=hd)
+    H.assert_quant_exact(r2["qact"], r2["ascales"], q_ref, a_ref, "w2 quant")
+    H.assert_y_close(r2["y"], y_ref, "w2")
+    H.assert_lowrank_close(r2["lowrank"], L_ref, "w2 L")
 
 
 @pytest.mark.parametrize("M,K,R", [(300, 512, 128), (64, 1024, 0), (1000, 2048, 128),
                                    (4352, 10240, 128)])
 def test_fused_silu_mul_quantize(M, K, R):
     # quantize_act of x = silu(a) * b, with x formed on chip: codes and
-    # scales identical to the unfused path (svdq_silu_mul, then
-    # svdq_quantize_act on its bf16 x), both equal to the oracle's on that
-    # x, and L within tolerance of the oracle.
+    # scales equal, bit for bit, to oracle.quantize_act(oracle.silu_mul(a,
+    # b)) on every row, and to the unfused path (svdq_silu_mul, then
+    # svdq_quantize_act); L within tolerance of the oracle's on that x.
     s = H.svdq()
     g = torch.Generator().manual_seed(M + K + R)
-    a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16).cuda()
-    b = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
-    sm = (torch.rand(K, generator=g) * 1.5 + 0.5).to(torch.bfloat16).cuda()
-    pd = (torch.randn(K, 128, generator=g) * 0.02).to(torch.bfloat16).cuda() if R else None
-    q1, a1, l1 = s.silu_mul_quantize_act(a, b, sm, pd)
-    h = s.silu_mul(a, b)
-    q2, a2, l2 = s.quantize_act(h, sm, pd)
+    a = (torch.randn(M, K, generator=g) * 2).to(torch.bfloat16)
+    b = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    sm = (torch.rand(K, generator=g) * 1.5 + 0.5).to(torch.bfloat16)
+    pd = (torch.randn(K, 128, generator=g) * 0.02).to(torch.bfloat16) if R else None
+    ad, bd, smd = a.cuda(), b.cuda(), sm.cuda()
+    pdd = pd.cuda() if R else None
+    q1, a1, l1 = s.silu_mul_quantize_act(ad, bd, smd, pdd)
+    h = s.silu_mul(ad, bd)
+    q2, a2, l2 = s.quantize_act(h, smd, pdd)
     s.check_device_error()
-    assert torch.equal(q1, q2)
+    h_ref = oracle.silu_mul(H.bits(a), H.bits(b))
+    assert np.array_equal(H.bits(h.cpu()), h_ref), "silu(a) * b differs from the oracle"
+    q_ref, a_ref = ref.quantize_act(h_ref, H.bits(sm))
     asc1 = s.unpack_scales(a1, M, K).cpu()
+    H.assert_quant_exact(q1.cpu(), asc1, q_ref, a_ref, "fused silu quant vs oracle")
+    assert torch.equal(q1, q2)
     assert torch.equal(asc1, s.unpack_scales(a2, M, K).cpu())
-    rows = H.sample_rows(M, 64, seed=K)
-    hc = h.cpu()
-    q_ref, a_ref = H.oracle_quant(hc[rows], sm.cpu())
-    H.assert_quant_exact(q1.cpu()[rows], asc1[rows], q_ref, a_ref, "fused silu quant")
     if R:
-        L_ref = ref.lowrank_down(H.bits(hc[rows]), H.bits(pd.cpu()))
-        H.assert_lowrank_close(l1.cpu()[rows], L_ref, "fused silu L")
+        L_ref = ref.lowrank_down(h_ref, H.bits(pd))
+        H.assert_lowrank_close(l1.cpu(), L_ref, "fused silu L")
     else:
         assert l1 is None
 
 
 def test_full_size_ffn_chain_fused():
-    # w1, w3, then w2 with its input formed on chip from their outputs.
+    # w1, w3, then w2 with its input formed on chip from their outputs;
+    # the oracle forms that input with its own silu_mul.
     s = H.svdq()
     names = ("ffn_w1_m4352_k3840_n10240", "ffn_w3_m4352_k3840_n10240", "ffn_w2_m4352_k10240_n3840")
     L1, L3, L2 = (synth.make_layer(*synth.WORKLOADS[n], seed=synth.workload_seed(n)) for n in names)
@@ -410,23 +410,13 @@ def test_full_size_ffn_chain_fused():
     y = s.w4a4_linear(qa, asc, lr, d["qweight"], wt, d["wcscales"], d["wtscale"], d["proj_up"],
                       d["bias"])
     s.check_device_error()
-    h = s.silu_mul(y1, y3).cpu()
-    rows = H.sample_rows(L2.M, 24, seed=9)
-    y_ref, q_ref, a_ref, _ = H.oracle_y(L2, rows=rows, x=h)
-    H.assert_quant_exact(qa.cpu()[rows], s.unpack_scales(asc, L2.M, L2.K).cpu()[rows], q_ref,
-                         a_ref, "fused w2 quant")
-    H.assert_y_close(y.cpu()[rows], y_ref, "fused w2")
-
-
-def test_silu_mul_tail_and_values():
-    s = H.svdq()
-    g = torch.Generator().manual_seed(3)
-    for n in (1, 7, 8, 9, 1000, 4097):
-        a = torch.randn(n, generator=g).to(torch.bfloat16)
-        b = torch.randn(n, generator=g).to(torch.bfloat16)
-        out = s.silu_mul(a.cuda(), b.cuda()).cpu()
-        want = (a.float() * torch.sigmoid(a.float()) * b.float())
-        assert ((out.float() - want).abs() <= 2 ** -7 * want.abs() + 1e-6).all(), n
+    h_ref = oracle.silu_mul(H.bits(r1["y"]), H.bits(r3["y"]))
+    h = torch.from_numpy(h_ref.view(np.int16)).view(torch.bfloat16)
+    y_ref, q_ref, a_ref, L_ref = H.oracle_y(L2, x=h)
+    H.assert_quant_exact(qa.cpu(), s.unpack_scales(asc, L2.M, L2.K).cpu(), q_ref, a_ref,
+                         "fused w2 quant")
+    H.assert_y_close(y.cpu(), y_ref, "fused w2")
+    H.assert_lowrank_close(lr.cpu(), L_ref, "fused w2 L")
 
 
 # ------------------------------------------------ seeded shape sweep ---
@@ -495,3 +485,172 @@ def test_small_m_transposed_gemm(M, K, N):
     p = H.gpu_plain_layer(L, True)
     yp, _, _ = H.oracle_plain_y(L, True)
     H.assert_y_close(p["y"], yp, f"plain {M}x{K}x{N}")
+
+
+# --------------------------------- every bf16 amax through the quantizer ---
+
+_E2M1_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+
+
+def _amax_sweep_groups(random_smooth: bool, seed: int):
+    """One 16-element group per positive finite bf16 value A: A itself (the
+    group's amax, at a rotating position and with alternating sign) and
+    the seven E2M1 midpoints of the group's scale d = e4m3(A / 6), both
+    signs, so that every element quotient is a tie.  With random smooth the
+    stored x is bf16(target / smooth), so v = x * smooth is a 16-bit product
+    next to the target instead of on it (targets up to 2^126, so that x
+    stays finite)."""
+    amax_bits = np.arange(1, 0x7F80, dtype=np.uint16)
+    A = nv.bf16_bits_to_f64(amax_bits)
+    if random_smooth:
+        # x = A / smooth must stay finite in bf16 and x * smooth in fp32
+        A = A[A <= 2.0 ** 126]
+    d = nv.decode_e4m3(nv.encode_e4m3_rne_satfinite(A / 6.0))
+    n = len(A)
+    G = np.zeros((n, 16))
+    mids = np.array(_E2M1_MIDPOINTS)
+    body = np.concatenate([mids[None, :] * d[:, None], -mids[None, :] * d[:, None],
+                           np.zeros((n, 1))], axis=1)                   # 15 values
+    body = np.minimum(np.abs(body), A[:, None]) * np.sign(body)         # keep A the amax
+    pos = np.arange(n) % 16
+    sign = np.where(np.arange(n) % 2 == 0, 1.0, -1.0)
+    for i in range(n):
+        row = list(body[i])
+        row.insert(pos[i], sign[i] * A[i])
+        G[i] = row
+    K = 64
+    rows = (n + 3) // 4
+    X = np.zeros((rows * 4, 16))
+    X[:n] = G
+    X = X.reshape(rows, K)
+    rng = np.random.default_rng(seed)
+    if random_smooth:
+        sm = torch.from_numpy(rng.uniform(0.5, 2.0, K)).to(torch.bfloat16)
+        x = (torch.from_numpy(X) / sm.double()[None, :]).to(torch.bfloat16)
+    else:
+        sm = torch.ones(K, dtype=torch.bfloat16)
+        x = torch.from_numpy(X).to(torch.bfloat16)
+        assert torch.equal(x.double(), torch.from_numpy(X)), "planted values must be bf16"
+    return x, sm
+
+
+@pytest.mark.parametrize("random_smooth", [False, True])
+def test_quantizer_every_bf16_amax_with_planted_ties(random_smooth):
+    # The activation kernel's divisions (reciprocal + one residual step)
+    # against the oracle's exact rounding, for every positive finite bf16
+    # value as a group amax, on the chip that runs them.
+    s = H.svdq()
+    x, sm = _amax_sweep_groups(random_smooth, seed=41)
+    M, K = x.shape
+    for R in (128, 0):
+        pd = torch.zeros(K, 128, dtype=torch.bfloat16).cuda() if R else None
+        qact, asc, _ = s.quantize_act(x.cuda(), sm.cuda(), pd)
+        s.check_device_error()
+        q_ref, a_ref = H.oracle_quant(x, sm)
+        H.assert_quant_exact(qact.cpu(), s.unpack_scales(asc, M, K).cpu(), q_ref, a_ref,
+                             f"amax sweep, random smooth {random_smooth}, R={R}")
+
+
+# ---------------------------- ragged K ranges and cluster-sum boundaries ---
+
+@pytest.mark.parametrize("M,K", [(16, 64 * 37), (64, 64 * 45), (100, 64 * 41), (200, 64 * 23),
+                                 (33, 64 * 161)])
+def test_quantize_ragged_k_split(M, K):
+    # K/64 not a multiple of the plan's split: the K ranges of a tile
+    # differ by 64 k and the last stage of some ranges holds one chunk.
+    s = H.svdq()
+    bm, split = s.quantize_plan(M, K)
+    assert split > 1 and (K // 64) % split != 0, (M, K, bm, split)
+    L = synth.make_layer(M, K, 32, seed=M + K)
+    qact, asc, lr = s.quantize_act(L.x.cuda(), L.smooth.cuda(), L.proj_down.cuda())
+    s.check_device_error()
+    q_ref, a_ref = H.oracle_quant(L.x, L.smooth)
+    H.assert_quant_exact(qact.cpu(), s.unpack_scales(asc, M, K).cpu(), q_ref, a_ref,
+                         f"ragged split M={M} K={K}")
+    H.assert_lowrank_close(lr.cpu(), ref.lowrank_down(H.bits(L.x), H.bits(L.proj_down)),
+                           f"ragged split L M={M} K={K}")
+
+
+@pytest.mark.parametrize("M,K,N", [(16, 256 * 5, 1024), (64, 256 * 7, 896), (1, 256 * 11, 1280),
+                                   (40, 256 * 13, 2048), (64, 256 * 37, 512)])
+def test_few_token_gemm_ragged_k_split(M, K, N):
+    # num_k = K/256 not a multiple of the few-token GEMM's cluster split:
+    # ranks hold different numbers of K steps, and the rank-order sum of
+    # the partials covers uneven ranges.
+    s = H.svdq()
+    kernel, split, grid = s.linear_plan(M, N, K)
+    assert kernel == s.GEMM_FEW_TOKENS and split > 1 and (K // 256) % split != 0, \
+        (M, N, K, kernel, split)
+    L = synth.make_layer(M, K, N, seed=M * 5 + K + N)
+    r = H.gpu_layer(L)
+    y_ref, q_ref, a_ref, _ = H.oracle_y(L)
+    H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, f"{M}x{K}x{N}")
+    H.assert_y_close(r["y"], y_ref, f"ragged few-token {M}x{K}x{N} split {split}")
+    p = H.gpu_plain_layer(L, True)
+    yp, _, _ = H.oracle_plain_y(L, True)
+    H.assert_y_close(p["y"], yp, f"plain ragged few-token {M}x{K}x{N}")
+
+
+def test_linear_plans_follow_their_rules():
+    # The launch shapes the host picks (not a restatement of them): the
+    # kernel by M (few tokens, single-SM tiles, CTA pairs), the few-token K
+    # split within 1..8, at most one K step short per rank, the clusters of
+    # a split in one wave.
+    s = H.svdq()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for M in (1, 16, 63, 64, 65, 256, 4352):
+        for N in (32, 416, 3840, 11520, 20480):
+            for K in (256, 768, 1280, 3840, 10240):
+                kernel, split, grid = s.linear_plan(M, N, K)
+                if M <= 64:
+                    assert kernel == s.GEMM_FEW_TOKENS
+                    n_tiles = -(-N // 128)
+                    assert split in (1, 2, 4, 8) and split <= K // 256
+                    if split > 1:
+                        assert grid == n_tiles * split <= sms
+                    else:
+                        assert grid == min(n_tiles, sms)
+                elif M <= 128:
+                    tiles = -(-M // 128) * -(-N // 256)
+                    assert kernel == s.GEMM_TOKEN_MAJOR and split == 1
+                    assert grid == min(tiles, sms)
+                else:
+                    # CTA pairs: an even grid, one pair per 256 x 256 tile
+                    # up to the pairs the device co-schedules
+                    tiles = -(-M // 256) * -(-N // 256)
+                    assert kernel == s.GEMM_PAIRS and split == 1
+                    assert grid % 2 == 0 and grid // 2 <= min(tiles, sms // 2)
+                    assert grid // 2 == tiles or grid >= sms - 2
+
+
+# ------------------------------------------------ concurrent repacks ---
+
+def test_concurrent_repacks_report_their_own_bad_scales():
+    # Two host threads repack at once on their own streams; one input has a
+    # sign-bit scale byte.  The bad-scale counter is shared per device, so
+    # the calls are serialized inside the library: the bad input must
+    # always give SVDQ_ERR_INVALID_ARG and the good one SVDQ_OK.
+    import threading
+    s = H.svdq()
+    good = torch.full((240, 3840), 0x38, dtype=torch.uint8).cuda()
+    bad = good.clone()
+    bad[117, 2000] = 0x80
+    results = {"good": [], "bad": []}
+
+    def worker(name, ws):
+        st = torch.cuda.Stream()
+        for _ in range(40):
+            try:
+                s.repack_weights(ws, stream=st)
+                results[name].append(s.SVDQ_OK)
+            except s.SvdqError as e:
+                results[name].append(e.status)
+
+    ts = [threading.Thread(target=worker, args=("good", good)),
+          threading.Thread(target=worker, args=("bad", bad))]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert results["good"] == [s.SVDQ_OK] * 40
+    assert results["bad"] == [s.SVDQ_ERR_INVALID_ARG] * 40
