@@ -288,23 +288,25 @@ def gemm_roofline(M, bytes_kg, flops_kg, kg_avg_ms, hbm_gbs, fp4_tflops, peak_sr
                               "FP4:BF16 dense ratio)",
                "algorithmic_flops_per_launch": flops_kg}
     out.update({"avg_launch_ms": round(kg_avg_ms, 5),
-                "timing": "CUDA events around each launch on its stream, second pass "
-                          "of the timed steps"})
+                "timing": "CUDA events on its stream around a run of the kernel alone, launched "
+                          "back to back over the timed steps' inputs; average per launch"})
     return out
 
 
-def run_step(svdq, d, stream, ev=None):
-    if ev is not None:
-        ev[0].record(stream)
+def run_kq(svdq, d, stream):
     svdq.quantize_act(d["x"], d["smooth"], d["proj_down"], qact=d["qact"], ascales_tiled=d["asc"],
                       lowrank=d["lr"], stream=stream)
-    if ev is not None:
-        ev[1].record(stream)
+
+
+def run_kg(svdq, d, stream):
     svdq.w4a4_linear(d["qact"], d["asc"], d["lr"], d["qweight"], d["wscales_tiled"],
                      d["wcscales"], d["wtscale"], d["proj_up"], d["bias"], y=d["y"],
                      stream=stream)
-    if ev is not None:
-        ev[2].record(stream)
+
+
+def run_step(svdq, d, stream):
+    run_kq(svdq, d, stream)
+    run_kg(svdq, d, stream)
 
 
 def bench_ours(args, world, rank, local):
@@ -338,7 +340,6 @@ def bench_ours(args, world, rank, local):
         svdq.check_device_error(stream)
 
         K_steps = args.steps
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
         clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
@@ -353,12 +354,21 @@ def bench_ours(args, world, rank, local):
         end.record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
-        # Per-kernel durations: a second pass over the same K steps with an
-        # event before, between and after the two kernels of each step
-        # (the events cost time of their own, so the step time above is
-        # taken without them).
+        # Per-kernel durations: each kernel alone, launched back to back over
+        # the same K steps' inputs (rotating sets), between two events; the
+        # average is its launch duration in a stream of its own launches.
+        # (Events between the kernels of every step would add the launch
+        # gap after each event to the kernel's time.)
+        kq_e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        kg_e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        kq_e[0].record(stream)
         for i in range(K_steps):
-            run_step(svdq, sets[i % nsets], stream, evs[i])
+            run_kq(svdq, sets[i % nsets], stream)
+        kq_e[1].record(stream)
+        kg_e[0].record(stream)
+        for i in range(K_steps):
+            run_kg(svdq, sets[i % nsets], stream)
+        kg_e[1].record(stream)
         torch.cuda.synchronize(dev)
         # The same steps from a CUDA graph (one step per rotating set,
         # captured once, replayed): what the kernels take without the
@@ -393,10 +403,8 @@ def bench_ours(args, world, rank, local):
         svdq.check_device_error(stream)
 
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
-    kq_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    kg_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    kq_avg = sum(kq_ms) / K_steps
-    kg_avg = sum(kg_ms) / K_steps
+    kq_avg = kq_e[0].elapsed_time(kq_e[1]) / K_steps
+    kg_avg = kg_e[0].elapsed_time(kg_e[1]) / K_steps
 
     value = job_value(one, K_steps, world, elapsed_ms)
     peaks, peak_src = load_peaks()
