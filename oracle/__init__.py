@@ -19,6 +19,11 @@ What it computes, and from which passage:
   (E2M1 elements with one e4m3 scale per 16 elements along K, R = 128).
 * The E2M1 bit layout (1 sign, 2 exponent, 1 mantissa bit) of the
   Z-Image NVFP4 blog, section "NVFP4 技术背景 / 什么是 NVFP4？".
+* The offline weight side (``weight_quant``): a bf16 weight and smoothing
+  factor to the stored operands through a rank-R SVD of the smoothed weight
+  and an NVFP4 residual -- the card's "via SVDQuant ... with rank-128 SVD
+  residual"; how the operands are derived is not on the pages, so each step
+  there is a reading stated in that module.
 * The input of the w2 feed-forward linear, silu(w1 x) * (w3 x), for the
   feed-forward linears w1, w2, w3 the same blog names in "Z-Image NVFP4
   模型变体" (``silu_mul``; the gated form is the reading taken).
@@ -40,6 +45,7 @@ from .nvfp4 import (  # noqa: F401
     pack_nibbles,
     unpack_nibbles,
 )
+from . import weight_quant  # noqa: F401
 from .svdq_ref import (  # noqa: F401
     quantize_act,
     lowrank_down,
