@@ -70,7 +70,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 8
+#define SVDQ_ABI_VERSION 9
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -186,6 +186,43 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
                      const uint16_t* wtscale, const uint16_t* proj_up,
                      const uint16_t* bias, int M, int N, int K, int R,
                      uint16_t* y, int ldy, void* stream);
+
+/* ---- offline weight side ------------------------------------------------ */
+
+/* Workspace svdq_quantize_weights needs for N output channels: (N + 1)
+ * floats.  0 on bad arguments. */
+size_t svdq_weight_workspace_bytes(int N);
+
+/* NVFP4 encoding of a weight's residual after its low-rank part, done once
+ * at load time (model card "nunchaku-z-image-turbo-svdq", first paragraph:
+ * "via SVDQuant, in NVFP4 ... with rank-128 SVD residual"; the operands of
+ * "What's stored on disk").  The pages do not say how the operands are
+ * derived; this call implements the reading
+ *   res[n, k]   = (W[n, k] - lowrank[n, k]) / smooth[k]
+ *   wtscale     = bf16(A / 2688), A = max |res|        (bf16 1 if A == 0)
+ *   wcscales[n] = bf16(a_n / A), a_n = max_k |res[n, k]| (0 if A == 0)
+ *   per 16 k:   wscales[k/16, n] = e4m3(a_g / (6 wtscale wcscales[n])),
+ *               qweight codes = E2M1(res / (wscales value * wtscale *
+ *               wcscales[n])), signed zero codes where that scale is 0,
+ * every float step a correctly rounded float32 operation in that order,
+ * every encoding nearest-even and saturating.  lowrank is the low-rank
+ * part proj_up @ proj_down^T of the caller's factors (a rank-R SVD of
+ * W / smooth, see svdq.py quantize_weights), so that the layer computes
+ * x @ W^T as closely as the formats allow.
+ *   W          [N, K] bf16, device; K % 16 == 0.
+ *   smooth     [K] bf16, device (all ones: no smoothing).
+ *   lowrank    [N, K] float32, device, or NULL (no low-rank part).
+ *   qweight    out, [N, K/2] bytes (low nibble = even k).
+ *   wscales    out, [K/16, N] e4m3 codes (the on-disk layout).
+ *   wcscales   out, [N] bf16;  wtscale out, [1] bf16.
+ *   workspace  device, svdq_weight_workspace_bytes(N) bytes, caller-owned;
+ *              overwritten.
+ * Inputs must be finite.  Enqueues three operations on `stream` (a 4-byte
+ * memset of the workspace and two kernels); returns SVDQ_OK, or a status
+ * for bad arguments. */
+int svdq_quantize_weights(const uint16_t* W, const uint16_t* smooth, const float* lowrank, int N,
+                          int K, uint8_t* qweight, uint8_t* wscales, uint16_t* wcscales,
+                          uint16_t* wtscale, void* workspace, void* stream);
 
 /* ---- helpers ------------------------------------------------------------ */
 

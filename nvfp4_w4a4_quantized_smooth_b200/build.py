@@ -23,7 +23,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libsvdq.so")
 SOURCES = ["svdq.cu"]
 HEADERS = ["sm100_ptx.cuh", "kq_quantize_act.cuh", "kg_w4a4_linear.cuh",
-           "kg2_w4a4_linear_pair.cuh", "ks_w4a4_linear_small.cuh", "kr_scales.cuh"]
+           "kg2_w4a4_linear_pair.cuh", "ks_w4a4_linear_small.cuh", "kr_scales.cuh",
+           "kw_quantize_weights.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -16,6 +16,7 @@
 #include "kg2_w4a4_linear_pair.cuh"
 #include "ks_w4a4_linear_small.cuh"
 #include "kr_scales.cuh"
+#include "kw_quantize_weights.cuh"
 
 namespace {
 
@@ -835,6 +836,39 @@ int svdq_silu_mul(const uint16_t* a, const uint16_t* b, uint16_t* out, size_t n,
                               static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const __nv_bfloat16*>(a), reinterpret_cast<const __nv_bfloat16*>(b),
       reinterpret_cast<__nv_bfloat16*>(out), n);
+  return launch_status();
+}
+
+size_t svdq_weight_workspace_bytes(int N) {
+  if (N < 1) return 0;
+  return (static_cast<size_t>(N) + 1) * sizeof(float);
+}
+
+int svdq_quantize_weights(const uint16_t* W, const uint16_t* smooth, const float* lowrank, int N,
+                          int K, uint8_t* qweight, uint8_t* wscales, uint16_t* wcscales,
+                          uint16_t* wtscale, void* workspace, void* stream) {
+  if (!W || !smooth || !qweight || !wscales || !wcscales || !wtscale || !workspace)
+    return SVDQ_ERR_INVALID_ARG;
+  if (N < 1 || K < 16 || K % 16) return SVDQ_ERR_SHAPE;
+  if (!aligned(W, 16) || !aligned(smooth, 2) || (lowrank && !aligned(lowrank, 16)) ||
+      !aligned(qweight, 8) || !aligned(wcscales, 2) || !aligned(wtscale, 2) ||
+      !aligned(workspace, 4))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  if (cudaMemsetAsync(ws + N, 0, sizeof(float), s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  const int rows_grid = N < d->num_sms * 8 ? N : d->num_sms * 8;
+  svdq::kw::weight_residual_amax_kernel<<<rows_grid, 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(W), lowrank,
+      reinterpret_cast<const __nv_bfloat16*>(smooth), N, K, ws);
+  if (launch_status()) return SVDQ_ERR_CUDA;
+  const size_t groups = static_cast<size_t>(N) * (K / 16);
+  svdq::kw::weight_quantize_kernel<<<grid_for(groups, 256, d->num_sms), 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(W), lowrank,
+      reinterpret_cast<const __nv_bfloat16*>(smooth), N, K, ws, qweight, wscales,
+      reinterpret_cast<__nv_bfloat16*>(wcscales), reinterpret_cast<__nv_bfloat16*>(wtscale));
   return launch_status();
 }
 

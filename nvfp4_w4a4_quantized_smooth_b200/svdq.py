@@ -29,7 +29,7 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 8
+ABI_VERSION = 9
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
 GEMM_TOKEN_MAJOR = 0
@@ -55,6 +55,8 @@ SIGNATURES = {
                               ctypes.POINTER(_I)]),
     "svdq_unpack_scales": (_I, [_P, _I, _I, _I, _P, _P]),
     "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
+    "svdq_weight_workspace_bytes": (_SZ, [_I]),
+    "svdq_quantize_weights": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
     "svdq_check_device_error": (_I, [_P]),
     "svdq_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
     "svdq_wait_probe": (_I, [_I, _P]),
@@ -283,6 +285,70 @@ def silu_mul(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = Non
         out = torch.empty_like(a)
     _check(_lib.svdq_silu_mul(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream(stream)),
            "svdq_silu_mul")
+    return out
+
+
+def quantize_weights_residual(W: torch.Tensor, smooth: torch.Tensor,
+                              lowrank: Optional[torch.Tensor] = None, stream=None):
+    """NVFP4 encoding of (W - lowrank) / smooth (svdq_quantize_weights) ->
+    (qweight [N, K/2] uint8, wscales [K/16, N] uint8 e4m3 codes, wcscales
+    [N] bf16, wtscale [1] bf16)."""
+    _need(W, torch.bfloat16, "W", 2)
+    _need(smooth, torch.bfloat16, "smooth", 1)
+    W = W.contiguous()
+    smooth = smooth.contiguous()
+    if lowrank is not None:
+        _need(lowrank, torch.float32, "lowrank", 2)
+        lowrank = lowrank.contiguous()
+    N, K = W.shape
+    dev = W.device
+    qweight = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+    wscales = torch.empty(K // 16, N, dtype=torch.uint8, device=dev)
+    wcscales = torch.empty(N, dtype=torch.bfloat16, device=dev)
+    wtscale = torch.empty(1, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(_lib.svdq_weight_workspace_bytes(N), dtype=torch.uint8, device=dev)
+    _check(_lib.svdq_quantize_weights(_ptr(W), _ptr(smooth), _ptr(lowrank), N, K, _ptr(qweight),
+                                      _ptr(wscales), _ptr(wcscales), _ptr(wtscale), _ptr(ws),
+                                      _stream(stream)),
+           "svdq_quantize_weights")
+    return qweight, wscales, wcscales, wtscale
+
+
+def quantize_weights(W: torch.Tensor, smooth: torch.Tensor, R: int = 128, stream=None,
+                     return_lowrank: bool = False):
+    """Offline weight side of the layer: a bf16 weight [N, K] and its
+    smoothing factor [K] -> the stored operands (a dict: qweight, wscales,
+    wcscales, wtscale, proj_down [K, R], proj_up [N, R]).
+
+    The low-rank factors are the rank-R truncated SVD of W / smooth
+    (proj_up = U_R S_R^1/2, proj_down = diag(smooth) V_R S_R^1/2, bf16),
+    computed with torch's linear algebra on the device (a library SVD and
+    GEMM: this runs once per layer at load time, not on the layer's path);
+    the residual and its NVFP4 encoding run in svdq_quantize_weights.
+    return_lowrank adds the float32 proj_up @ proj_down^T the encoding
+    used (for tests)."""
+    _need(W, torch.bfloat16, "W", 2)
+    _need(smooth, torch.bfloat16, "smooth", 1)
+    N, K = W.shape
+    if R > min(N, K):
+        raise ValueError("R exceeds the weight's rank bound")
+    s = smooth.float()
+    if R > 0:
+        U, S, Vh = torch.linalg.svd(W.float() / s[None, :], full_matrices=False)
+        sq = S[:R].sqrt()
+        proj_up = (U[:, :R] * sq[None, :]).to(torch.bfloat16).contiguous()
+        proj_down = (Vh[:R].T * sq[None, :] * s[:, None]).to(torch.bfloat16).contiguous()
+        lowrank = proj_up.float() @ proj_down.float().T
+    else:
+        proj_up = torch.zeros(N, 0, dtype=torch.bfloat16, device=W.device)
+        proj_down = torch.zeros(K, 0, dtype=torch.bfloat16, device=W.device)
+        lowrank = None
+    qweight, wscales, wcscales, wtscale = quantize_weights_residual(W, smooth, lowrank,
+                                                                    stream=stream)
+    out = dict(qweight=qweight, wscales=wscales, wcscales=wcscales, wtscale=wtscale,
+               proj_down=proj_down, proj_up=proj_up)
+    if return_lowrank:
+        out["lowrank"] = lowrank
     return out
 
 

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(svdq):
 
 
 def test_abi_version_and_status_strings(svdq):
-    assert svdq.abi_version() == 8 == svdq.ABI_VERSION
+    assert svdq.abi_version() == 9 == svdq.ABI_VERSION
     for st in range(8):
         s = svdq._lib.svdq_status_string(st).decode()
         assert s.startswith("SVDQ")
@@ -59,6 +59,8 @@ def test_size_queries(svdq):
     assert svdq.wscales_tiled_bytes(11520, 3840) == 90 * 60 * 512
     assert svdq.wscales_tiled_bytes(100, 64) == 2 * 1 * 512
     assert svdq.lowrank_bytes(4352, 128) == 4352 * 128 * 2
+    assert svdq._lib.svdq_weight_workspace_bytes(11520) == 11521 * 4
+    assert svdq._lib.svdq_weight_workspace_bytes(0) == 0
     for bad in ((0, 64), (16, 32), (16, 100)):
         assert svdq.ascales_tiled_bytes(*bad) == 0
         assert svdq.wscales_tiled_bytes(*bad) == 0
@@ -119,6 +121,20 @@ def test_argument_checks_fail_before_any_device_work(svdq):
                                           fake, None) == svdq.SVDQ_ERR_SHAPE
     assert lib.svdq_silu_mul_quantize_act(fake, odd, 16, 64, 64, fake, fake, 128, fake, fake,
                                           fake, None) == svdq.SVDQ_ERR_ALIGNMENT
+    # the offline weight quantizer: lowrank may be null, the rest may not;
+    # K a multiple of 16; 16-byte aligned W and lowrank
+    assert lib.svdq_quantize_weights(fake, fake, None, 32, 64, fake, fake, fake, fake, None,
+                                     None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_quantize_weights(None, fake, None, 32, 64, fake, fake, fake, fake, fake,
+                                     None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_quantize_weights(fake, fake, None, 32, 40, fake, fake, fake, fake, fake,
+                                     None) == svdq.SVDQ_ERR_SHAPE
+    assert lib.svdq_quantize_weights(fake, fake, None, 0, 64, fake, fake, fake, fake, fake,
+                                     None) == svdq.SVDQ_ERR_SHAPE
+    assert lib.svdq_quantize_weights(odd, fake, None, 32, 64, fake, fake, fake, fake, fake,
+                                     None) == svdq.SVDQ_ERR_ALIGNMENT
+    assert lib.svdq_quantize_weights(fake, fake, P(0x1004), 32, 64, fake, fake, fake, fake, fake,
+                                     None) == svdq.SVDQ_ERR_ALIGNMENT
     # scale unpack: only the two documented tile orders
     for kind in (-1, 2):
         assert lib.svdq_unpack_scales(fake, 16, 64, kind, fake, None) == svdq.SVDQ_ERR_INVALID_ARG
