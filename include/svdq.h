@@ -70,7 +70,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 9
+#define SVDQ_ABI_VERSION 10
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -223,6 +223,29 @@ size_t svdq_weight_workspace_bytes(int N);
 int svdq_quantize_weights(const uint16_t* W, const uint16_t* smooth, const float* lowrank, int N,
                           int K, uint8_t* qweight, uint8_t* wscales, uint16_t* wcscales,
                           uint16_t* wtscale, void* workspace, void* stream);
+
+/* The same encoding as svdq_quantize_weights for callers that cannot
+ * allocate device memory: code that runs inside a host framework or
+ * memory pool which owns all device memory and gives it no allocator, or
+ * a latency-critical thread that must not call cudaMalloc (which can
+ * synchronize the device).  The pages have no counterpart of this call; it
+ * only changes where the scratch lives.
+ * The row and global amax words live in one array that the library defines
+ * in device memory for at most 32768 output channels (128 KB on every
+ * device that loads the library, held until the process exits); N above
+ * that gives SVDQ_ERR_UNSUPPORTED and enqueues nothing.  The call
+ * allocates nothing: it enqueues a 4-byte memset of the array's global
+ * word (the one word that must start at zero; the rest keeps the previous
+ * call's values until overwritten) and the two kernels.  The first call on
+ * a device also looks up the array's device address on that device
+ * (cudaGetSymbolAddress) and keeps it; make that first call before any
+ * stream capture begins.  Every call on a device shares the array, so
+ * calls that overlap on the GPU (other streams, or other host threads
+ * without ordering) race on it: order them, e.g. on one stream.
+ * Arguments, outputs and statuses otherwise as svdq_quantize_weights. */
+int svdq_quantize_weights_noalloc(const uint16_t* W, const uint16_t* smooth, const float* lowrank,
+                                  int N, int K, uint8_t* qweight, uint8_t* wscales,
+                                  uint16_t* wcscales, uint16_t* wtscale, void* stream);
 
 /* ---- helpers ------------------------------------------------------------ */
 

@@ -872,6 +872,67 @@ int svdq_quantize_weights(const uint16_t* W, const uint16_t* smooth, const float
   return launch_status();
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of svdq_quantize_weights_noalloc: the per-row and global amax
+// words that svdq_quantize_weights keeps in its caller's workspace.  One
+// copy per device that loads the library, held until the process exits.
+constexpr int kNoAllocMaxRows = 32768;
+static __device__ __align__(256) float g_noalloc_weight_scratch[kNoAllocMaxRows + 1];
+
+// Device address of that array for each device, looked up once (with the
+// device current) on the first call there.  In host code the array's name
+// only stands for the symbol; it is not a device address.
+std::mutex g_noalloc_mu;
+float* g_noalloc_scratch_addr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" {
+
+int svdq_quantize_weights_noalloc(const uint16_t* W, const uint16_t* smooth, const float* lowrank,
+                                  int N, int K, uint8_t* qweight, uint8_t* wscales,
+                                  uint16_t* wcscales, uint16_t* wtscale, void* stream) {
+  if (!W || !smooth || !qweight || !wscales || !wcscales || !wtscale) return SVDQ_ERR_INVALID_ARG;
+  if (N < 1 || K < 16 || K % 16) return SVDQ_ERR_SHAPE;
+  if (N > kNoAllocMaxRows) return SVDQ_ERR_UNSUPPORTED;
+  if (!aligned(W, 16) || !aligned(smooth, 2) || (lowrank && !aligned(lowrank, 16)) ||
+      !aligned(qweight, 8) || !aligned(wcscales, 2) || !aligned(wtscale, 2))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  float* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_scratch_addr[dev] == nullptr) {
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_noalloc_weight_scratch) != cudaSuccess || addr == nullptr)
+        return SVDQ_ERR_CUDA;
+      g_noalloc_scratch_addr[dev] = static_cast<float*>(addr);
+    }
+    ws = g_noalloc_scratch_addr[dev];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The global amax word must start at zero; the per-row words are written
+  // before they are read.  Earlier calls' values are otherwise left in place.
+  if (cudaMemsetAsync(ws + N, 0, sizeof(float), s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  const int rows_grid = N < d->num_sms * 8 ? N : d->num_sms * 8;
+  svdq::kw::weight_residual_amax_kernel<<<rows_grid, 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(W), lowrank,
+      reinterpret_cast<const __nv_bfloat16*>(smooth), N, K, ws);
+  if (launch_status()) return SVDQ_ERR_CUDA;
+  const size_t groups = static_cast<size_t>(N) * (K / 16);
+  svdq::kw::weight_quantize_kernel<<<grid_for(groups, 256, d->num_sms), 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(W), lowrank,
+      reinterpret_cast<const __nv_bfloat16*>(smooth), N, K, ws, qweight, wscales,
+      reinterpret_cast<__nv_bfloat16*>(wcscales), reinterpret_cast<__nv_bfloat16*>(wtscale));
+  return launch_status();
+}
+
 int svdq_check_device_error(void* stream) {
   DeviceInfo* d = nullptr;
   if (int st = device_setup(&d)) return st;

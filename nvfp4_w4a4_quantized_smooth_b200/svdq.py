@@ -29,7 +29,7 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 9
+ABI_VERSION = 10
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
 GEMM_TOKEN_MAJOR = 0
@@ -57,6 +57,7 @@ SIGNATURES = {
     "svdq_silu_mul": (_I, [_P, _P, _P, _SZ, _P]),
     "svdq_weight_workspace_bytes": (_SZ, [_I]),
     "svdq_quantize_weights": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "svdq_quantize_weights_noalloc": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _P]),
     "svdq_check_device_error": (_I, [_P]),
     "svdq_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
     "svdq_wait_probe": (_I, [_I, _P]),

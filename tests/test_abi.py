@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(svdq):
 
 
 def test_abi_version_and_status_strings(svdq):
-    assert svdq.abi_version() == 9 == svdq.ABI_VERSION
+    assert svdq.abi_version() == 10 == svdq.ABI_VERSION
     for st in range(8):
         s = svdq._lib.svdq_status_string(st).decode()
         assert s.startswith("SVDQ")
