@@ -246,11 +246,23 @@ def make_sets(M, K, N, nsets, seed, dev, plain=False):
         d["repack_s"] = time.perf_counter() - t0
         e1.synchronize()
         d["repack_gpu_ms"] = e0.elapsed_time(e1)
+        d["proj_up_folded"] = None
+        d["fold_gpu_ms"] = 0.0
+        if not plain:
+            # the up-projection folded into the accumulator's units, once
+            # per weight (kept unfolded if some element does not fold)
+            e0.record()
+            folded, bad = svdq.fold_proj_up(d["proj_up"], d["wcscales"], d["wtscale"])
+            e1.record()
+            e1.synchronize()
+            d["fold_gpu_ms"] = e0.elapsed_time(e1)
+            d["proj_up_folded"] = folded if bad == 0 else None
         d["qact"] = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
         d["asc"] = torch.empty(svdq.ascales_tiled_bytes(M, K), dtype=torch.uint8, device=dev)
         d["lr"] = torch.empty(M, R, dtype=torch.bfloat16, device=dev)
         if plain:       # R = 0, no smoothing
             d["smooth"] = d["proj_down"] = d["proj_up"] = d["lr"] = None
+            d["proj_up_folded"] = None
         d["y"] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         sets.append(d)
     return sets
@@ -301,7 +313,7 @@ def run_kq(svdq, d, stream):
 def run_kg(svdq, d, stream):
     svdq.w4a4_linear(d["qact"], d["asc"], d["lr"], d["qweight"], d["wscales_tiled"],
                      d["wcscales"], d["wtscale"], d["proj_up"], d["bias"], y=d["y"],
-                     stream=stream)
+                     stream=stream, proj_up_folded=d["proj_up_folded"])
 
 
 def run_step(svdq, d, stream):
@@ -332,6 +344,8 @@ def bench_ours(args, world, rank, local):
     sets = probe + make_sets(M, K, N, nsets - 1, seed + 1, dev, plain)
     repack_us = 1e6 * statistics.median(d["repack_s"] for d in sets)
     repack_gpu_us = 1e3 * statistics.median(d["repack_gpu_ms"] for d in sets)
+    fold_gpu_us = 1e3 * statistics.median(d["fold_gpu_ms"] for d in sets)
+    folded = all(d["proj_up_folded"] is not None for d in sets)
 
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
@@ -443,6 +457,11 @@ def bench_ours(args, world, rank, local):
                          f"{per_set / 2**20:.0f} MiB",
                    "repack_us": round(repack_us, 1),
                    "repack_gpu_us": round(repack_gpu_us, 1),
+                   "lowrank_form": ("folded: proj_up / (wtscale * wcscales) prepared once per "
+                                    "weight by svdq_fold_proj_up, the low-rank product "
+                                    "accumulated with the block-scaled one" if folded else
+                                    "separate accumulator" if not plain else "none (R = 0)"),
+                   "fold_gpu_us": round(fold_gpu_us, 1),
                    "repack_timing": ("repack_us: host wall time of svdq_repack_weights, which "
                                      "synchronizes to read back the bad-scale count; "
                                      "repack_gpu_us: CUDA events around the call on its "
@@ -505,7 +524,7 @@ def bench_e2e(args, svdq, d, dev, M, K, N, world, r=R):
                               ascales_tiled=d["asc"], lowrank=d["lr"], stream=s_cmp)
             svdq.w4a4_linear(d["qact"], d["asc"], d["lr"], d["qweight"], d["wscales_tiled"],
                              d["wcscales"], d["wtscale"], d["proj_up"], d["bias"], y=y_dev[b],
-                             stream=s_cmp)
+                             stream=s_cmp, proj_up_folded=d["proj_up_folded"])
         cmp_done[b].record(s_cmp)
         s_d2h.wait_event(cmp_done[b])
         with torch.cuda.stream(s_d2h):
@@ -588,7 +607,8 @@ def bench_stack(args, world, rank, local):
             svdq.quantize_act(x, w.smooth, w.proj_down, qact=qa, ascales_tiled=asc, lowrank=lr,
                               stream=stream)
             svdq.w4a4_linear(qa, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
-                             w.proj_up, w.bias, y=y, stream=stream)
+                             w.proj_up, w.bias, y=y, stream=stream,
+                             proj_up_folded=w.proj_up_folded)
 
         hbuf = torch.empty_like(ybuf["w1"]) if args.unfused_w2 else None
 
@@ -605,7 +625,8 @@ def bench_stack(args, world, rank, local):
                 svdq.silu_mul_quantize_act(ybuf["w1"], ybuf["w3"], w.smooth, w.proj_down,
                                            qact=qa, ascales_tiled=asc, lowrank=lr, stream=stream)
             svdq.w4a4_linear(qa, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
-                             w.proj_up, w.bias, y=y, stream=stream)
+                             w.proj_up, w.bias, y=y, stream=stream,
+                             proj_up_folded=w.proj_up_folded)
 
         def step(evs=None):
             j = 0

@@ -70,7 +70,7 @@ typedef enum svdq_status {
 const char* svdq_status_string(int status);
 
 /* ABI version of this header (bumped on any signature change). */
-#define SVDQ_ABI_VERSION 10
+#define SVDQ_ABI_VERSION 11
 int svdq_abi_version(void);
 
 /* ---- size queries (bytes the caller allocates) ------------------------ */
@@ -166,8 +166,21 @@ int svdq_silu_mul_quantize_act(const uint16_t* a, const uint16_t* b, int M, int 
  *   wscales_tiled  as written by svdq_repack_weights.
  *   wcscales [N], wtscale [1] (read on the device), proj_up [N, R],
  *   bias [N] or NULL: bf16.
- *   R              128, or 0 without the low-rank branch (then lowrank and
- *                  proj_up are not used and may be NULL; the term is 0).
+ *   proj_up_folded NULL, or svdq_fold_proj_up's output for these proj_up,
+ *                  wcscales and wtscale, with no unfoldable element (the
+ *                  caller checks the count).  When given, the GEMM for
+ *                  M > 128 accumulates the low-rank product in the units
+ *                  of the block-scaled one, in the same fp32 accumulator:
+ *                    y = (acc + lowrank @ proj_up_folded^T) * wtscale
+ *                        * wcscales[n] + bias,
+ *                  the same value up to the bf16 rounding of the folded
+ *                  factor (relative 2^-9 per element, against the 2^-9 of
+ *                  proj_up's own bf16 storage), which lets that GEMM skip
+ *                  the second accumulator and its drain.  Other token
+ *                  counts use proj_up.  16-byte aligned.
+ *   R              128, or 0 without the low-rank branch (then lowrank,
+ *                  proj_up and proj_up_folded are not used and may be
+ *                  NULL; the term is 0).
  *   y              out, [M, ldy] bf16, ldy >= N, ldy % 8 == 0.
  * Limits: R in {0, 128}, K % 256 == 0, N % 32 == 0 (else
  * SVDQ_ERR_UNSUPPORTED).
@@ -184,8 +197,33 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled,
                      const uint16_t* lowrank, const uint8_t* qweight,
                      const void* wscales_tiled, const uint16_t* wcscales,
                      const uint16_t* wtscale, const uint16_t* proj_up,
-                     const uint16_t* bias, int M, int N, int K, int R,
-                     uint16_t* y, int ldy, void* stream);
+                     const uint16_t* proj_up_folded, const uint16_t* bias,
+                     int M, int N, int K, int R, uint16_t* y, int ldy,
+                     void* stream);
+
+/* One-time preparation of the up-projection for svdq_w4a4_linear's folded
+ * low-rank form (no counterpart on the pages: it re-associates the model
+ * card's runtime formula, "What's stored on disk", so that the low-rank
+ * product joins the block-scaled accumulator):
+ *   proj_up_folded[n, r] = bf16(proj_up[n, r] / (wtscale * wcscales[n])),
+ * the product wtscale * wcscales[n] exact in float32, the quotient
+ * correctly rounded to float32, then rounded to nearest-even bf16.
+ *   proj_up         [N, R] bf16, device, 16-byte aligned; R % 8 == 0.
+ *   wcscales [N], wtscale [1]: bf16, device.
+ *   proj_up_folded  out, [N, R] bf16, device, 16-byte aligned.
+ *   unfoldable      out, one uint32 in device memory: the number of
+ *                   elements that cannot be folded without losing
+ *                   precision (a zero or non-finite wtscale * wcscales[n],
+ *                   a quotient that is infinite or nonzero below the
+ *                   smallest normal bf16).  Zeroed by the call.  When it
+ *                   is not 0, do not pass proj_up_folded to
+ *                   svdq_w4a4_linear.
+ * Enqueues a 4-byte memset and one kernel on `stream`; returns SVDQ_OK or
+ * a status for bad arguments. */
+int svdq_fold_proj_up(const uint16_t* proj_up, const uint16_t* wcscales,
+                      const uint16_t* wtscale, int N, int R,
+                      uint16_t* proj_up_folded, uint32_t* unfoldable,
+                      void* stream);
 
 /* ---- offline weight side ------------------------------------------------ */
 

@@ -16,38 +16,55 @@
 // K steps in flight.
 //
 // Roles per CTA (both CTAs run all roles; only the even CTA issues MMAs):
-//   warp 0      producer (one thread).  A ring of STAGES stages; a stage
-//               holds one K step: this CTA's A rows (qact, 128 x 128 B) and
+//   warps 0, 10 producers (one thread each, taking the stage uses in
+//               turn).  A ring of STAGES stages; a stage holds one K step:
+//               this CTA's A rows (qact, 128 x 128 B) and
 //               B rows (qweight, 128 x 128 B) -- their TMA completions go
 //               to the even CTA's full barrier -- and the K step's scale
 //               blocks: this CTA's 128 A rows (2 KB) and all 256 B rows of
 //               the tile (4 KB: every CTA's TMEM needs all of the tile's B
 //               scales), bulk copies completing on this CTA's sf_loaded
-//               barrier.  After a tile's K steps two more stage uses carry
-//               the low-rank operands (a 64-wide half of R each: this CTA's
-//               L rows in the A place, its proj_up rows in the B place).
+//               barrier.  Two more stage uses per tile carry the low-rank
+//               operands (a 64-wide half of R each: this CTA's L rows in
+//               the A place, its proj_up rows in the B place), after the K
+//               steps (LR_SEPARATE) or before them (LR_FOLDED).
 //   warp 1      TMEM (512 columns, allocated for the pair); in the even CTA
 //               the MMA issuer: tcgen05.mma cta_group::2 kind::mxf4nvf4
 //               block16 (M = N = 256, K = 64, four per K step) into the main
-//               accumulator, then kind::f16 (K = 16) for L @ proj_up^T into
-//               the low-rank accumulator; its commits reach both CTAs.
+//               accumulator, and kind::f16 (K = 16) for the low-rank
+//               product; its commits reach both CTAs.
 //   warps 2..9  scale writers during the K loop and epilogue after it, in
 //               each CTA on its own TMEM (two warps per lane quarter):
 //               each stage's 12 scale blocks are written into that stage's
 //               TMEM scale slot with tcgen05.st (every block replicated in
 //               the four lane quarters, as the block-scaled MMA reads them),
-//               and the even CTA's sf_full barrier counts the 16 warps of
-//               the pair.  Epilogue: TMEM -> registers, fp32
-//               acc * wtscale * wcscales + lowrank + bias, bf16, TMEM
-//               released (to the even CTA), rows through a swizzled per-warp
+//               and each of the 16 warps of the pair arrives on the even
+//               CTA's full barrier of the stage.  Epilogue: TMEM -> registers, TMEM released (to
+//               the even CTA), fp32 acc * wtscale * wcscales (+ low-rank
+//               accumulator) + bias, bf16, rows through a swizzled per-warp
 //               shared-memory buffer to TMA tensor stores.
-// TMEM map (each CTA, 512 columns, fp32): main accumulator [0, 256),
-// low-rank accumulator [256, 512); the STAGES scale slots (48 columns each)
-// live in [256, 496) during the K loop.  Stage use u writes slot u % STAGES
-// only after the MMAs of use u - STAGES completed (the producer reloads the
-// stage's scale bytes only then), and a tile's first scale slots are
-// written only after every epilogue warp of the CTA has read the previous
-// tile's low-rank accumulator.
+// The low-rank branch takes one of two forms (template argument LRM):
+//   LR_SEPARATE  the formula's order: L @ proj_up^T in a second accumulator,
+//                added in the epilogue.  TMEM (each CTA, 512 fp32 columns):
+//                main accumulator [0, 256), low-rank accumulator [256, 512);
+//                the STAGES scale slots (48 columns each) live in
+//                [256, 496) during the K loop, so a tile's low-rank MMAs
+//                wait for its main MMAs (drain), and the next tile's first
+//                scale slots are written only after every epilogue warp of
+//                the CTA has read the low-rank accumulator.
+//   LR_FOLDED    proj_up_folded = bf16(proj_up / (wtscale * wcscales[n]))
+//                (prepared once per weight): the low-rank product is then in
+//                the units of the block-scaled one, and the two low-rank
+//                stage uses come first in the tile's K loop, into the main
+//                accumulator:  y = (acc + L proj_up_folded^T) * wtscale *
+//                wcscales[n] + bias.  TMEM: accumulator [0, 256), scale slots
+//                [256, 496) -- disjoint, so the scale writes run ahead of the
+//                epilogue, which reads the accumulator once and releases it
+//                before its arithmetic.
+//   LR_NONE      (R = 0) the folded form's schedule without low-rank uses.
+// In every form stage use u writes slot u % STAGES only after the MMAs of
+// use u - STAGES completed (the producer reloads the stage's scale bytes
+// only then).
 #pragma once
 
 #include <cuda.h>
@@ -78,7 +95,8 @@ static_assert(LR_A_BYTES <= A_BYTES && LR_B_BYTES <= B_BYTES, "low-rank halves f
 constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int EPI_WARP0 = 2;
-constexpr int NUM_THREADS = 32 * EPI_WARP0 + 32 * NUM_EPI_WARPS;
+constexpr int PROD1_WARP = EPI_WARP0 + NUM_EPI_WARPS;   // the second producer
+constexpr int NUM_THREADS = 32 * (PROD1_WARP + 1);
 constexpr int OUT_COLS = 64;                         // columns per TMA store box
 constexpr uint32_t OUT_WARP_BYTES = 32 * OUT_COLS * 2;   // 32 rows x 128 B
 constexpr uint32_t OUT_BYTES = NUM_EPI_WARPS * OUT_WARP_BYTES;
@@ -116,9 +134,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// LR: the layer has the low-rank branch (R = 128); without it (R = 0) a
-// tile has no low-rank stage uses, drain or MMAs.
-template <bool LR>
+// Low-rank forms (see the file comment).
+constexpr int LR_NONE = 0, LR_SEPARATE = 1, LR_FOLDED = 2;
+
+template <int LRM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/2] u8, box {128, 128}
                         const __grid_constant__ CUtensorMap tm_b,   // qweight [N, K/2] u8, box {128, 128}
@@ -136,14 +155,14 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
   const uint32_t s_out = s_ring + RING_BYTES;
   const uint32_t s_colv = s_out + OUT_BYTES;
   const uint32_t s_bar = s_colv + COLV_BYTES;
-  // Per stage: full (even CTA: both CTAs' operand bytes landed), empty (this
+  // Per stage: full (even CTA: both CTAs' operand bytes landed and all 16
+  // writer warps of the pair wrote the stage's scales into TMEM -- one
+  // barrier, so that the MMA thread waits once per stage use), empty (this
   // CTA: the stage's MMAs completed), sf_loaded (this CTA: its scale bytes
-  // landed), sf_full (even CTA: all 16 writer warps of the pair wrote the
-  // stage's scales into TMEM).
+  // landed).
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
   auto sfl_bar = [&](uint32_t s) { return s_bar + 8u * (2 * STAGES + s); };
-  auto sff_bar = [&](uint32_t s) { return s_bar + 8u * (3 * STAGES + s); };
   const uint32_t tmem_full_bar = s_bar + 8u * (4 * STAGES);
   const uint32_t tmem_empty_bar = tmem_full_bar + 8u;   // even CTA: 16 epilogue warps
   const uint32_t drain_bar = tmem_full_bar + 16u;
@@ -157,6 +176,8 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
   const uint32_t rank = cluster_ctarank();     // 0: the pair's MMA issuer
   const bool leader = rank == 0;
 
+  constexpr bool LR = LRM != LR_NONE;
+  constexpr bool FOLDED = LRM == LR_FOLDED;
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
@@ -166,10 +187,9 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
     }
     prefetch_tmap(&tm_y);
     for (uint32_t s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), 1 + 2 * NUM_EPI_WARPS);
       mbar_init(empty_bar(s), 1);
       mbar_init(sfl_bar(s), 1);
-      mbar_init(sff_bar(s), 2 * NUM_EPI_WARPS);
     }
     mbar_init(tmem_full_bar, 1);
     mbar_init(tmem_empty_bar, 2 * NUM_EPI_WARPS);
@@ -193,14 +213,26 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
 
   const int num_k = p.K / BK;                  // K steps per tile
   const int uses = num_k + (LR ? 2 : 0);       // stage uses per tile
+  // Position of a tile's first K step among its stage uses, and whether
+  // stage use `st` of a tile carries low-rank operands.
+  const int k0 = FOLDED ? 2 : 0;
+  auto lr_use = [&](int st) { return FOLDED ? st < 2 : (LR && st >= num_k); };
   const int tiles = p.m_tiles * p.n_tiles;
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
   const size_t kblocks = static_cast<size_t>(p.K / 64);   // 512-byte scale blocks per 128 rows
 
-  if (warp == 0) {
+  if (warp == 0 || warp == PROD1_WARP) {
     if (lane == 0) {
-      // ------------------------------------------------------ producer --
+      // ----------------------------------------------------- producers --
+      // Two producer threads in two warps take the stage uses in turn (one
+      // thread's copies complete about one stage per 0.3 us whatever the
+      // ring depth; two keep the SM's operand stream ahead of the MMAs).
+      // Each waits on a stage's empty barrier at most one phase ahead of
+      // its completion: its previous use waited for the release of the
+      // use STAGES + 2 back, and 2 <= STAGES.
+      static_assert(STAGES >= 2, "alternating producers need two stages");
+      const uint32_t pid = warp == 0 ? 0u : 1u;
       uint32_t it = 0;
       bool ok = true;
       for (int t = pair; t < tiles && ok; t += npairs) {
@@ -213,6 +245,7 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
         // operand box reads zeros; there is no scale block to copy.
         const bool a_sf = arow_tile < p.a_row_tiles;
         for (int st = 0; st < uses; ++st, ++it) {
+          if ((it & 1u) != pid) continue;
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!svdq_wait(empty_bar(s), ph ^ 1u, SITE_PROD)) {
@@ -220,20 +253,21 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
             break;
           }
           const uint32_t fb = map_to_rank(full_bar(s), 0);
-          if (st < num_k) {
+          if (!lr_use(st)) {
+            const int ks = st - k0;              // K step
             if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (A_BYTES + B_BYTES));
-            tma_load_2d_cg2(s_a(s), &tm_a, st * BK_BYTES, arow, fb);
-            tma_load_2d_cg2(s_b(s), &tm_b, st * BK_BYTES, brow, fb);
+            tma_load_2d_cg2(s_a(s), &tm_a, ks * BK_BYTES, arow, fb);
+            tma_load_2d_cg2(s_b(s), &tm_b, ks * BK_BYTES, brow, fb);
             mbar_arrive_expect_tx(sfl_bar(s), (a_sf ? SFA_BYTES : 0u) + SFB_BYTES);
             if (a_sf)
               bulk_load(s_sf(s),
-                        p.ascales_tiled + (static_cast<size_t>(arow_tile) * kblocks + 4 * st) * 512,
+                        p.ascales_tiled + (static_cast<size_t>(arow_tile) * kblocks + 4 * ks) * 512,
                         SFA_BYTES, sfl_bar(s));
             bulk_load(s_sf(s) + SFA_BYTES,
-                      p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * st) * 1024,
+                      p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * ks) * 1024,
                       SFB_BYTES, sfl_bar(s));
           } else {
-            const int hr = st - num_k;           // which 64-wide half of R
+            const int hr = FOLDED ? st : st - num_k;   // which 64-wide half of R
             if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (LR_A_BYTES + LR_B_BYTES));
             tma_load_2d_cg2(s_a(s), &tm_l, hr * 64, arow, fb);
             tma_load_2d_cg2(s_b(s), &tm_p, hr * 64, brow, fb);
@@ -250,6 +284,7 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
         const uint32_t n = it < STAGES ? it : STAGES;
         for (uint32_t j = 0; j < n; ++j) {
           const uint32_t jt = it - 1 - j;
+          if ((jt & 1u) != pid) continue;      // the other producer's use
           drain_wait(sfl_bar(jt % STAGES), (jt / STAGES) & 1u, 50000000ull);
           if (leader) drain_wait(full_bar(jt % STAGES), (jt / STAGES) & 1u, 50000000ull);
         }
@@ -265,28 +300,40 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
       for (int t = pair; t < tiles && ok; t += npairs, ++tc) {
         if (!svdq_wait(tmem_empty_bar, (tc & 1u) ^ 1u, SITE_MMA_TE)) break;
         tc_fence_after();
-        for (int st = 0; st < num_k; ++st, ++it) {
+        // LR_FOLDED: the two low-rank uses first (the first MMA starts the
+        // accumulator), then the K steps, all into the main accumulator.
+        const int main_uses = FOLDED ? uses : num_k;
+        for (int st = 0; st < main_uses; ++st, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
-          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL) ||
-              !svdq_wait(sff_bar(s), ph, SITE_MMA_SF)) {
+          if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
-          const uint32_t sfb_t = sfa_t + 16;
+          if (FOLDED && st < 2) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            mma_nvfp4_cg2(tmem_base + TM_ACC,
-                          smem_desc(s_a(s) + 32 * j, 16, 1024, kLayoutSwizzle128B),
-                          smem_desc(s_b(s) + 32 * j, 16, 1024, kLayoutSwizzle128B), idesc_main,
-                          sfa_t + 4 * j, sfb_t + 8 * j, (st | j) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_cg2(tmem_base + TM_ACC,
+                          smem_desc(s_a(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B),
+                          smem_desc(s_b(s) + 32 * kk, 16, 1024, kLayoutSwizzle128B), idesc_lr,
+                          (st | kk) != 0 ? 1u : 0u);
+          } else {
+            const uint32_t sfa_t = tmem_base + TM_SF + TM_SF_SLOT * s;
+            const uint32_t sfb_t = sfa_t + 16;
+            const int ks = st - k0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              mma_nvfp4_cg2(tmem_base + TM_ACC,
+                            smem_desc(s_a(s) + 32 * j, 16, 1024, kLayoutSwizzle128B),
+                            smem_desc(s_b(s) + 32 * j, 16, 1024, kLayoutSwizzle128B), idesc_main,
+                            sfa_t + 4 * j, sfb_t + 8 * j, (FOLDED || (ks | j) != 0) ? 1u : 0u);
+            }
           }
           tc_commit_cg2_mc(empty_bar(s), 0x3);
         }
         if (!ok) break;
-        if (LR) {
+        if (LRM == LR_SEPARATE) {
           // The low-rank accumulator overlaps the scale slots: every main
           // MMA completes before the low-rank MMAs write there.
           tc_commit_cg2(drain_bar);
@@ -295,8 +342,7 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
           for (int hr = 0; hr < 2 && ok; ++hr, ++it) {
             const uint32_t s = it % STAGES;
             const uint32_t ph = (it / STAGES) & 1u;
-            if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL) ||
-                !svdq_wait(sff_bar(s), ph, SITE_MMA_SF)) {
+            if (!svdq_wait(full_bar(s), ph, SITE_MMA_FULL)) {
               ok = false;
               break;
             }
@@ -325,7 +371,7 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
     const float alpha = __bfloat162float(p.wtscale[0]);
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const uint32_t s_obuf = s_out + static_cast<uint32_t>(warp - EPI_WARP0) * OUT_WARP_BYTES;
-    const uint32_t sff_leader0 = map_to_rank(sff_bar(0), 0);
+    const uint32_t full_leader0 = map_to_rank(full_bar(0), 0);
     const uint32_t tmem_empty_leader = map_to_rank(tmem_empty_bar, 0);
     float* wc_s = reinterpret_cast<float*>(smem + (s_colv - s_ring));
     float* bs_s = wc_s + BN;
@@ -342,7 +388,7 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
         const uint32_t ph = (u / STAGES) & 1u;
         if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(sfl_bar(s), ph, SITE_SF_LOADED));
         if (!ok) continue;
-        if (static_cast<int>(u % static_cast<uint32_t>(uses)) < num_k) {
+        if (!lr_use(static_cast<int>(u % static_cast<uint32_t>(uses)))) {
           const uint32_t src = s_sf(s) + 16 * lane;
           const uint32_t dst = lane_base + TM_SF + TM_SF_SLOT * s;
 #pragma unroll
@@ -357,75 +403,25 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
           tc_fence_before();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(sff_leader0 + 8u * s);
+        if (lane == 0) mbar_arrive_remote(full_leader0 + 8u * s);
       }
     };
-    // A tile's first `head` stage uses are written right after the previous
-    // tile's TMEM reads, before its output stores, and `mid` more between
-    // the two output pieces, so the MMAs restart soon and do not wait for
-    // the stores.
-    const uint32_t head = num_k < STAGES ? static_cast<uint32_t>(num_k) : STAGES;
-    const uint32_t mid = num_k - head < 2u ? num_k - head : 2u;
-    const uint32_t rest = static_cast<uint32_t>(uses) - head - mid;
-    if (pair < tiles) write_uses(head + mid);
-    for (int t = pair; t < tiles; t += npairs, ++tc) {
-      const int mb = t % p.m_tiles;
-      const int nb = t / p.m_tiles;
-      const bool has_next = t + npairs < tiles;
-      write_uses(rest);
-      // Per-column factors of this tile -> shared memory (every warp has
-      // finished the previous tile's arithmetic, which read them).
-      {
-        const int n = nb * BN + et;
-        float wcv = 0.f, bsv = 0.f;
-        if (n < p.N) {
-          wcv = __bfloat162float(p.wcscales[n]);
-          if (p.bias != nullptr) bsv = __bfloat162float(p.bias[n]);
-        }
-        wc_s[et] = wcv * alpha;
-        bs_s[et] = bsv;
+    // Per-column factors of tile column nb -> shared memory (every warp has
+    // finished the previous tile's arithmetic, which read them).
+    auto load_columns = [&](int nb) {
+      const int n = nb * BN + et;
+      float wcv = 0.f, bsv = 0.f;
+      if (n < p.N) {
+        wcv = __bfloat162float(p.wcscales[n]);
+        if (p.bias != nullptr) bsv = __bfloat162float(p.bias[n]);
       }
-      // Every epilogue warp passes the named barriers once per tile, also
-      // after a failed wait, so that no warp is left waiting on them.
-      named_bar_sync(2, 32 * NUM_EPI_WARPS);
-      if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI));
-      uint32_t out[8][8];
-      if (ok) {
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int col = half * 128 + 16 * c;
-          uint32_t acc[16], lr[16];
-          tmem_ld_32x32b_x16(lane_base + TM_ACC + col, acc);
-          if (LR) {
-            tmem_ld_32x32b_x16(lane_base + TM_LR + col, lr);
-          } else {
-#pragma unroll
-            for (int z = 0; z < 16; ++z) lr[z] = 0u;   // +0.0f
-          }
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float2 w2 = *reinterpret_cast<const float2*>(wc_s + col + 2 * i);
-            const float2 b2 = *reinterpret_cast<const float2*>(bs_s + col + 2 * i);
-            const float o0 = fmaf(__uint_as_float(acc[2 * i]), w2.x,
-                                  __uint_as_float(lr[2 * i]) + b2.x);
-            const float o1 = fmaf(__uint_as_float(acc[2 * i + 1]), w2.y,
-                                  __uint_as_float(lr[2 * i + 1]) + b2.y);
-            out[c][i] = pack_bf16x2(o0, o1);
-          }
-        }
-        tc_fence_before();
-      }
-      // All TMEM reads of this CTA are done: the low-rank columns (which the
-      // next tile's scale slots overlap) and the accumulator are free.
-      named_bar_sync(3, 32 * NUM_EPI_WARPS);
-      if (!ok) continue;
-      if (lane == 0) mbar_arrive_remote(tmem_empty_leader);
-      if (has_next) write_uses(head);
-      // Rows -> swizzled buffer (row = lane, 128 B per row; 16-byte chunk
-      // j of row r at chunk j ^ (r % 8), the TMA 128-byte swizzle) -> TMA
-      // store of 32 rows x 64 columns, twice per tile.
+      wc_s[et] = wcv * alpha;
+      bs_s[et] = bsv;
+    };
+    // Rows -> swizzled buffer (row = lane, 128 B per row; 16-byte chunk j of
+    // row r at chunk j ^ (r % 8), the TMA 128-byte swizzle) -> TMA store of
+    // 32 rows x 64 columns, twice per tile; `between` runs after the first.
+    auto store_rows = [&](const uint32_t (&out)[8][8], int mb, int nb, auto&& between) {
       const int row0 = mb * BM + static_cast<int>(rank) * BM_CTA + q * 32;
 #pragma unroll
       for (int pc = 0; pc < 2; ++pc) {
@@ -445,7 +441,123 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
           tma_store_2d(&tm_y, s_obuf, x0, row0);
           bulk_commit_group();
         }
-        if (pc == 0 && has_next) write_uses(mid);
+        if (pc == 0) between();
+      }
+    };
+    // Every epilogue warp passes the named barriers once per tile, also
+    // after a failed wait, so that no warp is left waiting on them.
+    if constexpr (LRM == LR_SEPARATE) {
+      // A tile's first `head` stage uses are written right after the
+      // previous tile's TMEM reads, before its output stores, and `mid` more
+      // between the two output pieces, so the MMAs restart soon and do not
+      // wait for the stores.
+      const uint32_t head = num_k < STAGES ? static_cast<uint32_t>(num_k) : STAGES;
+      const uint32_t mid = num_k - head < 2u ? num_k - head : 2u;
+      const uint32_t rest = static_cast<uint32_t>(uses) - head - mid;
+      if (pair < tiles) write_uses(head + mid);
+      for (int t = pair; t < tiles; t += npairs, ++tc) {
+        const int mb = t % p.m_tiles;
+        const int nb = t / p.m_tiles;
+        const bool has_next = t + npairs < tiles;
+        write_uses(rest);
+        load_columns(nb);
+        named_bar_sync(2, 32 * NUM_EPI_WARPS);
+        if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI));
+        uint32_t out[8][8];
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int col = half * 128 + 16 * c;
+            uint32_t acc[16], lr[16];
+            tmem_ld_32x32b_x16(lane_base + TM_ACC + col, acc);
+            tmem_ld_32x32b_x16(lane_base + TM_LR + col, lr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 w2 = *reinterpret_cast<const float2*>(wc_s + col + 2 * i);
+              const float2 b2 = *reinterpret_cast<const float2*>(bs_s + col + 2 * i);
+              const float o0 = fmaf(__uint_as_float(acc[2 * i]), w2.x,
+                                    __uint_as_float(lr[2 * i]) + b2.x);
+              const float o1 = fmaf(__uint_as_float(acc[2 * i + 1]), w2.y,
+                                    __uint_as_float(lr[2 * i + 1]) + b2.y);
+              out[c][i] = pack_bf16x2(o0, o1);
+            }
+          }
+          tc_fence_before();
+        }
+        // All TMEM reads of this CTA are done: the low-rank columns (which
+        // the next tile's scale slots overlap) and the accumulator are free.
+        named_bar_sync(3, 32 * NUM_EPI_WARPS);
+        if (!ok) continue;
+        if (lane == 0) mbar_arrive_remote(tmem_empty_leader);
+        if (has_next) write_uses(head);
+        store_rows(out, mb, nb, [&] {
+          if (has_next) write_uses(mid);
+        });
+      }
+    } else {
+      // Scale slots and accumulator are disjoint, so the scale writes run
+      // ahead of the epilogue.  Of the next tile's stage uses, `pre` are
+      // written before this tile's accumulator is read (their stages land
+      // while this tile's last K steps run), `post` right after it is
+      // released, `mid` between the two output pieces and the rest after
+      // the stores.  Each warp releases the accumulator as soon as its own
+      // reads are done; the arithmetic follows.
+      const uint32_t U = static_cast<uint32_t>(uses);
+      const uint32_t pre = U < 3u ? U : 3u;
+      const uint32_t post = U - pre < 2u ? U - pre : 2u;
+      const uint32_t mid = U - pre - post < 2u ? U - pre - post : 2u;
+      const uint32_t rest = U - pre - post - mid;
+      if (pair < tiles) write_uses(U);
+      for (int t = pair; t < tiles; t += npairs, ++tc) {
+        const int mb = t % p.m_tiles;
+        const int nb = t / p.m_tiles;
+        const bool has_next = t + npairs < tiles;
+        load_columns(nb);
+        named_bar_sync(2, 32 * NUM_EPI_WARPS);
+        if (has_next) write_uses(pre);
+        if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI));
+        // Two batches of 64 columns (all 128 would not fit the registers
+        // beside the output words); the accumulator is released after the
+        // second batch's reads, before its arithmetic.
+        uint32_t out[8][8];
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t acc[4][16];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tmem_ld_32x32b_x16(lane_base + TM_ACC + half * 128 + 64 * h + 16 * c, acc[c]);
+            tmem_ld_wait();
+            if (h == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_remote(tmem_empty_leader);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int col = half * 128 + 64 * h + 16 * c;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float2 w2 = *reinterpret_cast<const float2*>(wc_s + col + 2 * i);
+                const float2 b2 = *reinterpret_cast<const float2*>(bs_s + col + 2 * i);
+                out[4 * h + c][i] =
+                    pack_bf16x2(fmaf(__uint_as_float(acc[c][2 * i]), w2.x, b2.x),
+                                fmaf(__uint_as_float(acc[c][2 * i + 1]), w2.y, b2.y));
+              }
+            }
+          }
+        }
+        if (has_next) write_uses(post);
+        // Every warp has read this tile's column factors.
+        named_bar_sync(3, 32 * NUM_EPI_WARPS);
+        if (!ok) continue;
+        store_rows(out, mb, nb, [&] {
+          if (has_next) write_uses(mid);
+        });
+        if (has_next) write_uses(rest);
       }
     }
     if (lane == 0) bulk_wait_group0();

@@ -81,6 +81,46 @@ __global__ void unpack_scales_kernel(const uint8_t* __restrict__ tiled, int rows
   }
 }
 
+// proj_up_folded[n, r] = bf16(proj_up[n, r] / (wtscale * wcscales[n])): the
+// up-projection in the units of the block-scaled product, so that
+//   (acc + L proj_up_folded^T) * wtscale * wcscales[n] + bias
+// is the layer's acc * wtscale * wcscales[n] + L proj_up^T + bias up to the
+// bf16 rounding of the folded factor (the float32 quotient, correctly
+// rounded, then rounded to nearest-even bf16).  An element that cannot be
+// folded without losing its precision -- a zero or non-finite scale, a
+// quotient that is infinite or below the smallest normal bf16 (and not zero)
+// -- is counted in *unfoldable.  One thread per 8 elements.
+__global__ void fold_proj_up_kernel(const __nv_bfloat16* __restrict__ proj_up,
+                                    const __nv_bfloat16* __restrict__ wcscales,
+                                    const __nv_bfloat16* __restrict__ wtscale, int N, int R,
+                                    __nv_bfloat16* __restrict__ out,
+                                    uint32_t* __restrict__ unfoldable) {
+  const float alpha = __bfloat162float(wtscale[0]);
+  const size_t total = static_cast<size_t>(N) * R / 8;
+  uint32_t bad = 0;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(i * 8 / R);
+    const float scale = __fmul_rn(alpha, __bfloat162float(wcscales[n]));
+    const bool scale_ok = scale != 0.0f && isfinite(scale);
+    const uint4 v = reinterpret_cast<const uint4*>(proj_up)[i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float q0 = __fdiv_rn(__uint_as_float(w[j] << 16), scale);
+      const float q1 = __fdiv_rn(__uint_as_float(w[j] & 0xFFFF0000u), scale);
+      const __nv_bfloat162 r = __floats2bfloat162_rn(q0, q1);
+      o[j] = *reinterpret_cast<const uint32_t*>(&r);
+      const float f0 = __low2float(r), f1 = __high2float(r);
+      bad += !scale_ok || !isfinite(f0) || (f0 != 0.0f && fabsf(f0) < 1.17549435e-38f);
+      bad += !scale_ok || !isfinite(f1) || (f1 != 0.0f && fabsf(f1) < 1.17549435e-38f);
+    }
+    reinterpret_cast<uint4*>(out)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (bad) atomicAdd(unfoldable, bad);
+}
+
 // out = silu(a) * b = a / (1 + exp(-a)) * b rounded once to bf16
 // (silu_mul_words: fp32 with an fp64 path near bf16 rounding boundaries).
 __global__ void silu_mul_kernel(const __nv_bfloat16* __restrict__ a,

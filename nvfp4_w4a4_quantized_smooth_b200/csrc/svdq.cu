@@ -99,10 +99,13 @@ int device_setup(DeviceInfo** out) {
           cudaFuncSetAttribute(ks::w4a4_linear_small_kernel<false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                ks::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(kg2::w4a4_linear_pair_kernel<true>,
+          cudaFuncSetAttribute(kg2::w4a4_linear_pair_kernel<kg2::LR_NONE>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kg2::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(kg2::w4a4_linear_pair_kernel<false>,
+          cudaFuncSetAttribute(kg2::w4a4_linear_pair_kernel<kg2::LR_SEPARATE>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kg2::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(kg2::w4a4_linear_pair_kernel<kg2::LR_FOLDED>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kg2::SMEM_BYTES) != cudaSuccess)
         return SVDQ_ERR_CUDA;
@@ -253,7 +256,9 @@ int kg2_max_pairs(DeviceInfo* d) {
   cfg.numAttrs = 1;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(
-          &n, reinterpret_cast<const void*>(svdq::kg2::w4a4_linear_pair_kernel<true>), &cfg) !=
+          &n, reinterpret_cast<const void*>(
+                  svdq::kg2::w4a4_linear_pair_kernel<svdq::kg2::LR_SEPARATE>),
+          &cfg) !=
       cudaSuccess) {
     cudaGetLastError();
     n = 0;
@@ -341,14 +346,17 @@ int launch_small(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
 }
 
 // The token-major GEMM on CTA pairs (kg2_w4a4_linear_pair.cuh), 256 x 256
-// tiles.  Arguments as checked by svdq_w4a4_linear.
+// tiles; the low-rank product in the main accumulator when the folded
+// up-projection is given.  Arguments as checked by svdq_w4a4_linear.
 int launch_pair(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
                 const uint16_t* lowrank, const uint8_t* qweight, const void* wscales_tiled,
                 const uint16_t* wcscales, const uint16_t* wtscale, const uint16_t* proj_up,
-                const uint16_t* bias, int M, int N, int K, int R, uint16_t* y, int ldy,
-                void* stream) {
+                const uint16_t* proj_up_folded, const uint16_t* bias, int M, int N, int K, int R,
+                uint16_t* y, int ldy, void* stream) {
   namespace kg2 = svdq::kg2;
   const bool lr = R != 0;
+  const bool folded = lr && proj_up_folded != nullptr;
+  if (folded) proj_up = proj_up_folded;
   const uint64_t kb = static_cast<uint64_t>(K) / 2;
   CUtensorMap tm_a, tm_b, tm_l, tm_p, tm_y;
   if (make_tmap(&tm_a, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, kg2::BK_BYTES,
@@ -395,10 +403,12 @@ int launch_pair(DeviceInfo* d, const uint8_t* qact, const void* ascales_tiled,
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   const cudaError_t e =
-      lr ? cudaLaunchKernelEx(&cfg, kg2::w4a4_linear_pair_kernel<true>, tm_a, tm_b, tm_l, tm_p,
-                              tm_y, p)
-         : cudaLaunchKernelEx(&cfg, kg2::w4a4_linear_pair_kernel<false>, tm_a, tm_b, tm_l, tm_p,
-                              tm_y, p);
+      folded ? cudaLaunchKernelEx(&cfg, kg2::w4a4_linear_pair_kernel<kg2::LR_FOLDED>, tm_a, tm_b,
+                                  tm_l, tm_p, tm_y, p)
+      : lr   ? cudaLaunchKernelEx(&cfg, kg2::w4a4_linear_pair_kernel<kg2::LR_SEPARATE>, tm_a,
+                                  tm_b, tm_l, tm_p, tm_y, p)
+             : cudaLaunchKernelEx(&cfg, kg2::w4a4_linear_pair_kernel<kg2::LR_NONE>, tm_a, tm_b,
+                                  tm_l, tm_p, tm_y, p);
   if (e != cudaSuccess) return SVDQ_ERR_CUDA;
   return launch_status();
 }
@@ -705,8 +715,9 @@ int svdq_silu_mul_quantize_act(const uint16_t* a, const uint16_t* b, int M, int 
 
 int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint16_t* lowrank,
                      const uint8_t* qweight, const void* wscales_tiled, const uint16_t* wcscales,
-                     const uint16_t* wtscale, const uint16_t* proj_up, const uint16_t* bias, int M,
-                     int N, int K, int R, uint16_t* y, int ldy, void* stream) {
+                     const uint16_t* wtscale, const uint16_t* proj_up,
+                     const uint16_t* proj_up_folded, const uint16_t* bias, int M, int N, int K,
+                     int R, uint16_t* y, int ldy, void* stream) {
   const bool lr = R != 0;
   if (!qact || !ascales_tiled || !qweight || !wscales_tiled || !wcscales || !wtscale || !y ||
       (lr && (!lowrank || !proj_up)))
@@ -715,7 +726,8 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
   if ((R != 128 && R != 0) || K % svdq::kg::BK || N % 32) return SVDQ_ERR_UNSUPPORTED;
   if (!aligned(qact, 16) || !aligned(ascales_tiled, 16) || !aligned(qweight, 16) ||
       !aligned(wscales_tiled, 16) || !aligned(wcscales, 16) || !aligned(wtscale, 2) ||
-      (lr && (!aligned(lowrank, 16) || !aligned(proj_up, 16))) || (bias && !aligned(bias, 16)) ||
+      (lr && (!aligned(lowrank, 16) || !aligned(proj_up, 16))) ||
+      (proj_up_folded && !aligned(proj_up_folded, 16)) || (bias && !aligned(bias, 16)) ||
       !aligned(y, 16) || ldy % 8)
     return SVDQ_ERR_ALIGNMENT;
   DeviceInfo* d = nullptr;
@@ -727,7 +739,7 @@ int svdq_w4a4_linear(const uint8_t* qact, const void* ascales_tiled, const uint1
                         wtscale, proj_up, bias, M, N, K, R, y, ldy, stream);
   if (M >= kPairMinM)
     return launch_pair(d, qact, ascales_tiled, lowrank, qweight, wscales_tiled, wcscales,
-                       wtscale, proj_up, bias, M, N, K, R, y, ldy, stream);
+                       wtscale, proj_up, proj_up_folded, bias, M, N, K, R, y, ldy, stream);
   CUtensorMap tm_a, tm_b, tm_l, tm_p, tm_y;
   if (make_tmap(&tm_a, qact, CU_TENSOR_MAP_DATA_TYPE_UINT8, kb, M, kb, svdq::kg::BK_BYTES,
                 svdq::kg::BM) ||
@@ -836,6 +848,29 @@ int svdq_silu_mul(const uint16_t* a, const uint16_t* b, uint16_t* out, size_t n,
                               static_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const __nv_bfloat16*>(a), reinterpret_cast<const __nv_bfloat16*>(b),
       reinterpret_cast<__nv_bfloat16*>(out), n);
+  return launch_status();
+}
+
+int svdq_fold_proj_up(const uint16_t* proj_up, const uint16_t* wcscales, const uint16_t* wtscale,
+                      int N, int R, uint16_t* proj_up_folded, uint32_t* unfoldable,
+                      void* stream) {
+  if (!proj_up || !wcscales || !wtscale || !proj_up_folded || !unfoldable)
+    return SVDQ_ERR_INVALID_ARG;
+  if (N < 1 || R < 1) return SVDQ_ERR_SHAPE;
+  if (R % 8) return SVDQ_ERR_UNSUPPORTED;
+  if (!aligned(proj_up, 16) || !aligned(proj_up_folded, 16) || !aligned(wcscales, 2) ||
+      !aligned(wtscale, 2) || !aligned(unfoldable, 4))
+    return SVDQ_ERR_ALIGNMENT;
+  DeviceInfo* d = nullptr;
+  if (int st = device_setup(&d)) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(unfoldable, 0, sizeof(uint32_t), s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  const size_t work = static_cast<size_t>(N) * R / 8;
+  svdq::kr::fold_proj_up_kernel<<<grid_for(work, 256, d->num_sms), 256, 0, s>>>(
+      reinterpret_cast<const __nv_bfloat16*>(proj_up),
+      reinterpret_cast<const __nv_bfloat16*>(wcscales),
+      reinterpret_cast<const __nv_bfloat16*>(wtscale), N, R,
+      reinterpret_cast<__nv_bfloat16*>(proj_up_folded), unfoldable);
   return launch_status();
 }
 

@@ -29,7 +29,7 @@ SVDQ_ERR_CUDA = 6
 SVDQ_ERR_TIMEOUT = 7
 
 # Constants of include/svdq.h.
-ABI_VERSION = 10
+ABI_VERSION = 11
 SCALES_ACT = 0
 SCALES_WEIGHT = 1
 GEMM_TOKEN_MAJOR = 0
@@ -48,7 +48,9 @@ SIGNATURES = {
     "svdq_lowrank_bytes": (_SZ, [_I, _I]),
     "svdq_repack_weights": (_I, [_P, _I, _I, _P, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
-    "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P]),
+    "svdq_w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I,
+                              _P]),
+    "svdq_fold_proj_up": (_I, [_P, _P, _P, _I, _I, _P, _P, _P]),
     "svdq_silu_mul_quantize_act": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
     "svdq_quantize_plan": (_I, [_I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "svdq_linear_plan": (_I, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
@@ -218,10 +220,13 @@ def w4a4_linear(qact: torch.Tensor, ascales_tiled: torch.Tensor,
                 lowrank: Optional[torch.Tensor], qweight: torch.Tensor,
                 wscales_tiled: torch.Tensor, wcscales: torch.Tensor, wtscale: torch.Tensor,
                 proj_up: Optional[torch.Tensor], bias: Optional[torch.Tensor],
-                y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                y: Optional[torch.Tensor] = None, stream=None,
+                proj_up_folded: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The block-scaled FP4 GEMM with the fused epilogue -> y [M, N] bf16.
 
-    lowrank and proj_up None: the plain NVFP4 layer (R = 0)."""
+    lowrank and proj_up None: the plain NVFP4 layer (R = 0).  proj_up_folded:
+    fold_proj_up's factor for these proj_up / wcscales / wtscale (the GEMM
+    for M > 128 then adds the low-rank product inside its accumulator)."""
     _need(qact, torch.uint8, "qact", 2)
     _need(qweight, torch.uint8, "qweight", 2)
     if (lowrank is None) != (proj_up is None):
@@ -229,6 +234,10 @@ def w4a4_linear(qact: torch.Tensor, ascales_tiled: torch.Tensor,
     if lowrank is not None:
         _need(lowrank, torch.bfloat16, "lowrank", 2)
         _need(proj_up, torch.bfloat16, "proj_up", 2)
+    if proj_up_folded is not None:
+        _need(proj_up_folded, torch.bfloat16, "proj_up_folded", 2)
+        if proj_up is None or proj_up_folded.shape != proj_up.shape:
+            raise ValueError("proj_up_folded needs proj_up of the same shape")
     M = qact.shape[0]
     K = qact.shape[1] * 2
     N = qweight.shape[0]
@@ -237,10 +246,29 @@ def w4a4_linear(qact: torch.Tensor, ascales_tiled: torch.Tensor,
         y = torch.empty(M, N, dtype=torch.bfloat16, device=qact.device)
     _check(_lib.svdq_w4a4_linear(_ptr(qact), _ptr(ascales_tiled), _ptr(lowrank),
                                  _ptr(qweight), _ptr(wscales_tiled), _ptr(wcscales),
-                                 _ptr(wtscale), _ptr(proj_up), _ptr(bias), M, N, K, R,
-                                 _ptr(y), y.stride(0), _stream(stream)),
+                                 _ptr(wtscale), _ptr(proj_up), _ptr(proj_up_folded), _ptr(bias),
+                                 M, N, K, R, _ptr(y), y.stride(0), _stream(stream)),
            "svdq_w4a4_linear")
     return y
+
+
+def fold_proj_up(proj_up: torch.Tensor, wcscales: torch.Tensor, wtscale: torch.Tensor,
+                 stream=None):
+    """svdq_fold_proj_up -> (proj_up_folded [N, R] bf16, number of elements
+    that cannot be folded).  Reads the count back (synchronizes the
+    stream); pass the factor to w4a4_linear only when the count is 0."""
+    _need(proj_up, torch.bfloat16, "proj_up", 2)
+    N, R = proj_up.shape
+    out = torch.empty_like(proj_up)
+    count = torch.empty(1, dtype=torch.int32, device=proj_up.device)
+    _check(_lib.svdq_fold_proj_up(_ptr(proj_up), _ptr(wcscales), _ptr(wtscale), N, R, _ptr(out),
+                                  _ptr(count), _stream(stream)),
+           "svdq_fold_proj_up")
+    if stream is not None:
+        stream.synchronize()
+    else:
+        torch.cuda.current_stream(proj_up.device).synchronize()
+    return out, int(count.item())
 
 
 def quantize_plan(M: int, K: int):
@@ -369,12 +397,17 @@ def wait_probe(arrive: bool, stream=None) -> None:
 
 
 class PreparedWeights:
-    """One layer's device weights with the scales already repacked."""
+    """One layer's device weights with the scales already repacked and (fold
+    True, R > 0) the up-projection folded where every element folds."""
 
     def __init__(self, qweight, wscales, wcscales, wtscale, smooth, proj_down, proj_up,
-                 bias=None, stream=None):
+                 bias=None, stream=None, fold=True):
         self.qweight = qweight
         self.wscales_tiled = repack_weights(wscales, stream=stream)
+        self.proj_up_folded = None
+        if fold and proj_up is not None and proj_up.shape[1] > 0:
+            folded, bad = fold_proj_up(proj_up, wcscales, wtscale, stream=stream)
+            self.proj_up_folded = folded if bad == 0 else None
         self.wcscales = wcscales
         self.wtscale = wtscale
         self.smooth = smooth
@@ -390,4 +423,4 @@ def svdq_linear(x: torch.Tensor, w: PreparedWeights, y: Optional[torch.Tensor] =
     """Whole layer on device tensors: svdq_quantize_act then svdq_w4a4_linear."""
     qact, asc, lr = quantize_act(x, w.smooth, w.proj_down, stream=stream)
     return w4a4_linear(qact, asc, lr, w.qweight, w.wscales_tiled, w.wcscales, w.wtscale,
-                       w.proj_up, w.bias, y=y, stream=stream)
+                       w.proj_up, w.bias, y=y, stream=stream, proj_up_folded=w.proj_up_folded)

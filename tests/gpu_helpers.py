@@ -40,7 +40,10 @@ def to_dev(L: synth.LayerOperands, dev="cuda"):
 
 
 def gpu_layer(L: synth.LayerOperands, x_override=None):
-    """Run quantize + linear on the GPU; return CPU results."""
+    """Run quantize + linear on the GPU; return CPU results: y with the
+    low-rank product in its own accumulator (the formula's order) and
+    y_fold with the folded up-projection (fold_proj_up), the form the
+    CTA-pair GEMM (M > 128) takes it in; smaller M ignore the folded factor."""
     s = svdq()
     d = to_dev(L)
     if x_override is not None:
@@ -50,11 +53,15 @@ def gpu_layer(L: synth.LayerOperands, x_override=None):
     qact, asc, lr = s.quantize_act(d["x"], d["smooth"], d["proj_down"])
     y = s.w4a4_linear(qact, asc, lr, d["qweight"], wt, d["wcscales"], d["wtscale"],
                       d["proj_up"], d["bias"])
+    folded, bad = s.fold_proj_up(d["proj_up"], d["wcscales"], d["wtscale"])
+    assert bad == 0, f"{bad} up-projection elements do not fold"
+    y_fold = s.w4a4_linear(qact, asc, lr, d["qweight"], wt, d["wcscales"], d["wtscale"],
+                           d["proj_up"], d["bias"], proj_up_folded=folded)
     s.check_device_error()
     asc_logical = s.unpack_scales(asc, M, K)
     torch.cuda.synchronize()
     return dict(qact=qact.cpu(), ascales=asc_logical.cpu(), lowrank=lr.cpu(), y=y.cpu(),
-                wtiled=wt)
+                y_fold=y_fold.cpu(), wtiled=wt)
 
 
 def bits(t):

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(svdq):
 
 
 def test_abi_version_and_status_strings(svdq):
-    assert svdq.abi_version() == 10 == svdq.ABI_VERSION
+    assert svdq.abi_version() == 11 == svdq.ABI_VERSION
     for st in range(8):
         s = svdq._lib.svdq_status_string(st).decode()
         assert s.startswith("SVDQ")
@@ -73,8 +73,8 @@ def test_argument_checks_fail_before_any_device_work(svdq):
     # null pointers
     assert lib.svdq_quantize_act(None, 16, 64, 64, fake, fake, 128, fake, fake, fake,
                                  None) == svdq.SVDQ_ERR_INVALID_ARG
-    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 64,
-                                256, 128, None, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, None, 16,
+                                64, 256, 128, None, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_repack_weights(None, 64, 64, fake, None) == svdq.SVDQ_ERR_INVALID_ARG
     # shapes
     assert lib.svdq_quantize_act(fake, 0, 64, 64, fake, fake, 128, fake, fake, fake,
@@ -83,25 +83,38 @@ def test_argument_checks_fail_before_any_device_work(svdq):
                                  None) == svdq.SVDQ_ERR_SHAPE
     assert lib.svdq_quantize_act(fake, 16, 64, 32, fake, fake, 128, fake, fake, fake,
                                  None) == svdq.SVDQ_ERR_SHAPE
-    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 64,
-                                256, 128, fake, 32, None) == svdq.SVDQ_ERR_SHAPE
+    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, None, 16,
+                                64, 256, 128, fake, 32, None) == svdq.SVDQ_ERR_SHAPE
     # implemented limits
     assert lib.svdq_quantize_act(fake, 16, 64, 64, fake, fake, 64, fake, fake, fake,
                                  None) == svdq.SVDQ_ERR_UNSUPPORTED
     assert lib.svdq_quantize_act(fake, 16, 80, 80, fake, fake, 128, fake, fake, fake,
                                  None) == svdq.SVDQ_ERR_UNSUPPORTED
-    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 64,
-                                192, 128, fake, 64, None) == svdq.SVDQ_ERR_UNSUPPORTED
-    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, 16, 48,
-                                256, 128, fake, 48, None) == svdq.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, None, 16,
+                                64, 192, 128, fake, 64, None) == svdq.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, None, 16,
+                                48, 256, 128, fake, 48, None) == svdq.SVDQ_ERR_UNSUPPORTED
     # alignment
     odd = P(0x1001)
     assert lib.svdq_quantize_act(odd, 16, 64, 64, fake, fake, 128, fake, fake, fake,
                                  None) == svdq.SVDQ_ERR_ALIGNMENT
     assert lib.svdq_quantize_act(fake, 16, 64, 68, fake, fake, 128, fake, fake, fake,
                                  None) == svdq.SVDQ_ERR_ALIGNMENT
-    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, odd, 16, 64,
-                                256, 128, fake, 64, None) == svdq.SVDQ_ERR_ALIGNMENT
+    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, None, odd, 16,
+                                64, 256, 128, fake, 64, None) == svdq.SVDQ_ERR_ALIGNMENT
+    assert lib.svdq_w4a4_linear(fake, fake, fake, fake, fake, fake, fake, fake, odd, None, 16,
+                                64, 256, 128, fake, 64, None) == svdq.SVDQ_ERR_ALIGNMENT
+    # the folded up-projection: arguments, shape, R % 8, alignment
+    assert lib.svdq_fold_proj_up(None, fake, fake, 64, 128, fake, fake,
+                                 None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_fold_proj_up(fake, fake, fake, 64, 128, fake, None,
+                                 None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_fold_proj_up(fake, fake, fake, 0, 128, fake, fake,
+                                 None) == svdq.SVDQ_ERR_SHAPE
+    assert lib.svdq_fold_proj_up(fake, fake, fake, 64, 12, fake, fake,
+                                 None) == svdq.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_fold_proj_up(odd, fake, fake, 64, 128, fake, fake,
+                                 None) == svdq.SVDQ_ERR_ALIGNMENT
     # R = 0 (no low-rank branch): proj_down, lowrank, proj_up and smooth may
     # be null; the other checks still apply
     assert lib.svdq_quantize_act(fake, 0, 64, 64, None, None, 0, fake, fake, None,
@@ -110,10 +123,10 @@ def test_argument_checks_fail_before_any_device_work(svdq):
                                  None) == svdq.SVDQ_ERR_INVALID_ARG
     assert lib.svdq_quantize_act(fake, 16, 64, 64, None, None, 128, fake, fake, fake,
                                  None) == svdq.SVDQ_ERR_INVALID_ARG      # R = 128 needs proj_down
-    assert lib.svdq_w4a4_linear(fake, fake, None, fake, fake, fake, fake, None, None, 16, 48,
-                                256, 0, fake, 48, None) == svdq.SVDQ_ERR_UNSUPPORTED
-    assert lib.svdq_w4a4_linear(fake, fake, None, fake, fake, fake, fake, None, None, 16, 64,
-                                256, 128, fake, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
+    assert lib.svdq_w4a4_linear(fake, fake, None, fake, fake, fake, fake, None, None, None, 16,
+                                48, 256, 0, fake, 48, None) == svdq.SVDQ_ERR_UNSUPPORTED
+    assert lib.svdq_w4a4_linear(fake, fake, None, fake, fake, fake, fake, None, None, None, 16,
+                                64, 256, 128, fake, 64, None) == svdq.SVDQ_ERR_INVALID_ARG
     # the fused w2 activation: b is required, the other checks as quantize_act
     assert lib.svdq_silu_mul_quantize_act(fake, None, 16, 64, 64, fake, fake, 128, fake, fake,
                                           fake, None) == svdq.SVDQ_ERR_INVALID_ARG

@@ -205,6 +205,9 @@ def test_linear_parity(M, K, N):
     y_ref, q_ref, a_ref, _ = H.oracle_y(L)
     H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, "quant")
     H.assert_y_close(r["y"], y_ref, f"M={M} K={K} N={N}")
+    H.assert_y_close(r["y_fold"], y_ref, f"folded M={M} K={K} N={N}")
+    if M <= 128:   # only the CTA-pair GEMM takes the folded factor
+        assert torch.equal(r["y_fold"].view(torch.int16), r["y"].view(torch.int16))
 
 
 @pytest.mark.parametrize("M,K,N,with_smooth", [(300, 512, 384, False), (128, 1024, 512, True),
@@ -255,8 +258,9 @@ def test_integer_grid_invariant_bit_exact():
     r = H.gpu_layer(L)
     y_ref, *_ = H.oracle_y(L)
     want = nv.f64_to_bf16_bits_rne(y_ref)
-    got = H.bits(r["y"])
-    assert np.array_equal(got, want), f"{(got != want).sum()} outputs differ"
+    for key in ("y", "y_fold"):
+        got = H.bits(r[key])
+        assert np.array_equal(got, want), f"{key}: {(got != want).sum()} outputs differ"
 
 
 def test_unit_scales_random_codes_exact():
@@ -279,8 +283,9 @@ def test_unit_scales_random_codes_exact():
     r = H.gpu_layer(L)
     y_ref, *_ = H.oracle_y(L)
     want = nv.f64_to_bf16_bits_rne(y_ref)
-    got = H.bits(r["y"])
-    assert np.array_equal(got, want), f"{(got != want).sum()} outputs differ"
+    for key in ("y", "y_fold"):
+        got = H.bits(r[key])
+        assert np.array_equal(got, want), f"{key}: {(got != want).sum()} outputs differ"
 
 
 def test_zero_weights_give_lowrank_branch_only():
@@ -291,6 +296,7 @@ def test_zero_weights_give_lowrank_branch_only():
           @ oracle.bf16_bits_to_f64(H.bits(L.proj_up)).T
           + oracle.bf16_bits_to_f64(H.bits(L.bias)))
     H.assert_y_close(r["y"], lr, "low-rank only")
+    H.assert_y_close(r["y_fold"], lr, "low-rank only, folded")
 
 
 def test_output_row_stride():
@@ -319,6 +325,7 @@ def _full_size_check(name):
     y_ref, q_ref, a_ref, L_ref = H.oracle_y(L)
     H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, name)
     H.assert_y_close(r["y"], y_ref, name)
+    H.assert_y_close(r["y_fold"], y_ref, f"{name} folded")
     H.assert_lowrank_close(r["lowrank"], L_ref, name)
     return L, r
 
@@ -444,9 +451,11 @@ def test_shape_sweep_all_paths(M, K, N):
     y_ref, q_ref, a_ref, L_ref = H.oracle_y(L)
     H.assert_quant_exact(r["qact"], r["ascales"], q_ref, a_ref, f"layer {M}x{K}x{N}")
     H.assert_y_close(r["y"], y_ref, f"layer {M}x{K}x{N}")
+    H.assert_y_close(r["y_fold"], y_ref, f"folded layer {M}x{K}x{N}")
     H.assert_lowrank_close(r["lowrank"], L_ref, f"layer {M}x{K}x{N}")
     again = H.gpu_layer(L)
     assert torch.equal(again["y"].view(torch.int16), r["y"].view(torch.int16))
+    assert torch.equal(again["y_fold"].view(torch.int16), r["y_fold"].view(torch.int16))
     for with_smooth in (False, True):
         p = H.gpu_plain_layer(L, with_smooth)
         yp, qp, ap = H.oracle_plain_y(L, with_smooth)
