@@ -11,28 +11,28 @@
 //                                   satfinite conversion
 //   q = E2M1(v / s)                 quotient, then the hardware RNE /
 //                                   satfinite conversion
-// Each quotient a / b is formed as r = 1/b (reciprocal), q0 = a r, then one
-// residual step (Markstein, IBM J. Res. Dev. 34(1), 1990) with the residual
-// exact by FMA.  Rounding that q equals rounding the exact quotient: a
-// bf16 x bf16 product has at most 16 significant bits, and every e4m3
-// midpoint x 6 and every E2M1 midpoint x s at most 7, so a quotient that is
-// not exactly a midpoint lies at least 2^-16 (relative) from it, far more
-// than q's error (a few ulps of fp32); a quotient that is exactly a
-// midpoint is representable and the residual step returns it exactly
-// (|1 - b r| <= 2^-22 makes the step's error far below half an ulp), so the
-// conversion sees the tie.
-// The element quotients are computed on nv = x * (-smooth) = -v with the
-// negated reciprocal: q0 = nv (-r) = v r, e = q0 s + nv = q0 s - v,
-// q = q0 + e (-r).  These are the same roundings as q0 = v r,
-// e = v - q0 s, q = q0 + e r, and they also keep the sign of a zero v
-// (v = -0 gives q0 = -0, e = +0, q = -0; v = +0 gives +0), which the E2M1
-// code must carry.  A scale that rounds to zero gives -r = -0 and therefore
-// signed zero codes.
-//
+// The scale's quotient amax / 6 is one product with RN(1/6): a bf16 x bf16
+// product has at most 16 significant bits and every e4m3 midpoint x 6 at
+// most 7, so a quotient that is not exactly a midpoint lies at least 2^-16
+// (relative) from it, far more than the product's error; at an exact
+// midpoint t (at most 5 significant bits) the product is t (1 + 2^-25 or
+// so), within half an ulp of t, so it rounds to t and the conversion sees
+// the tie.
+// An element's quotient v / d takes the reciprocal in two parts: r_hi =
+// 1/d rounded down (__frcp_rd), r_lo = (1 - d r_hi) r_hi >= 0 (the residual
+// exact by FMA), and q = RN(v r_hi + RN(v r_lo)): within about 2^-46
+// (relative) of v / d, so non-midpoints round as the exact quotient does
+// (the same 2^-16 argument, the midpoints of E2M1 x d having at most 7
+// bits) and an exact midpoint comes out exactly.  Both parts are >= 0, so
+// the sign of a zero v is kept (v r_lo and v r_hi carry it, and zeros of
+// one sign add to that sign); a scale that rounds to zero gives r_hi =
+// r_lo = 0 and therefore signed zero codes.
+
 // CTA work item: a tile of BM rows (64 or 128, a template parameter) and
 // one of `split` ranges of K; the `split` CTAs of a tile form a
-// thread-block cluster.  18 warps:
-//   warp 0      TMA producer: per stage of 128 k, the x tile (one 3-D box:
+// thread-block cluster.  19 warps:
+//   warps 0, 18 TMA producers (taking the stages in turn): per stage of
+//               128 k, the x tile (one 3-D box:
 //               2 chunks x [BM rows x 64 k] bf16, 128-byte swizzle), the
 //               proj_down rows (one 3-D box: 2 halves of 64 r x [128 k x
 //               128 B]) and 256 B of smooth, into a ring of stages.
@@ -79,7 +79,8 @@ constexpr uint32_t PD_BYTES = 2 * PD_HALF;         // 32 KB
 constexpr uint32_t SM_BYTES = STAGE_K * 2;         // 256 B
 constexpr int NUM_QWARPS = 16;
 constexpr int NUM_QTHREADS = NUM_QWARPS * 32;
-constexpr int NUM_THREADS = 64 + NUM_QTHREADS;
+constexpr int PROD1_WARP = 2 + NUM_QWARPS;   // the second producer
+constexpr int NUM_THREADS = 64 + NUM_QTHREADS + 32;
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BUDGET = 227 * 1024;
 constexpr int PART_STRIDE = R + 4;     // floats per row of a staged partial (bank spread)
@@ -141,40 +142,39 @@ __device__ __forceinline__ uint64_t bf16x2_to_pk(uint32_t w) {
   return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
-// One 16-element group: x (8 bf16x2 words) and the negated smooth values
-// as packed fp32 pairs -> 16 E2M1 codes (element 0 in the lowest nibble)
-// and the e4m3 scale byte.
+// One 16-element group: x (8 bf16x2 words) and the smooth values as packed
+// fp32 pairs -> 16 E2M1 codes (element 0 in the lowest nibble) and the e4m3
+// scale byte.
 __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
-                                                   const uint64_t (&nsm)[8],
+                                                   const uint64_t (&sm2)[8],
                                                    uint32_t& scale_byte) {
-  uint64_t nv[8];
+  uint64_t v[8];
   float m8[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    nv[i] = mul2(bf16x2_to_pk(xw[i]), nsm[i]);
+    v[i] = mul2(bf16x2_to_pk(xw[i]), sm2[i]);
     float lo, hi;
-    upk(nv[i], lo, hi);
+    upk(v[i], lo, hi);
     m8[i] = fmaxf(fabsf(lo), fabsf(hi));
   }
   // max is exact, so a tree gives the same amax with a short dependency chain
   const float amax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                            fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-  // amax / 6 with one residual step; r6 = RN(1/6).
-  const float r6 = __uint_as_float(0x3E2AAAABu);
-  const float a0 = amax * r6;
-  const float a6 = fmaf(fmaf(-a0, 6.0f, amax), r6, a0);
-  const uint32_t sc = cvt_e4m3x2(a6, 0.0f) & 0xFFu;
+  const float r6 = __uint_as_float(0x3E2AAAABu);   // RN(1/6)
+  const uint32_t sc = cvt_e4m3x2(amax * r6, 0.0f) & 0xFFu;
   scale_byte = sc;
   const float d = e4m3_to_f32(sc);
-  const float nr = d > 0.0f ? -rcp_approx(d) : -0.0f;
-  const uint64_t nr2 = pk(nr, nr);
-  const uint64_t d2 = pk(d, d);
+  float r_hi = 0.0f, r_lo = 0.0f;
+  if (d > 0.0f) {
+    r_hi = __frcp_rd(d);
+    r_lo = fmaf(-d, r_hi, 1.0f) * r_hi;
+  }
+  const uint64_t rhi2 = pk(r_hi, r_hi);
+  const uint64_t rlo2 = pk(r_lo, r_lo);
   float q[16];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint64_t q0 = mul2(nv[i], nr2);       // v r
-    const uint64_t e = fma2(q0, d2, nv[i]);     // q0 s - v, exact
-    const uint64_t q1 = fma2(e, nr2, q0);       // q0 + (v - q0 s) r
+    const uint64_t q1 = fma2(v[i], rhi2, mul2(v[i], rlo2));
     upk(q1, q[2 * i], q[2 * i + 1]);
   }
   const float(&qlo)[8] = *reinterpret_cast<const float(*)[8]>(q);
@@ -250,12 +250,17 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
 
   bool l_ready = false;   // quantizer threads: L^T accumulator readable
 
-  if (warp == 0) {
+  if (warp == 0 || warp == PROD1_WARP) {
     if (lane == 0) {
-      // ------------------------------------------------------ producer --
-      int i = 0;
+      // ----------------------------------------------------- producers --
+      // Two threads in two warps take the stages in turn (one thread's
+      // copies complete about one stage per 0.3 us whatever the ring
+      // depth); each waits on a stage's empty barrier at most one phase
+      // ahead of its completion, as 2 <= STAGES.
+      const int pid = warp == 0 ? 0 : 1;
+      int i = pid;
       bool ok = true;
-      for (; i < nstages; ++i) {
+      for (; i < nstages; i += 2) {
         const uint32_t s = static_cast<uint32_t>(i) % STAGES;
         const uint32_t ph = (static_cast<uint32_t>(i) / STAGES) & 1u;
         if (!svdq_wait(empty_bar(s), ph ^ 1u, SITE_PROD)) {
@@ -277,6 +282,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
         const int n = i < STAGES ? i : STAGES;
         for (int j = 0; j < n; ++j) {
           const uint32_t jt = static_cast<uint32_t>(i - 1 - j);
+          if (static_cast<int>(jt & 1u) != pid) continue;   // the other producer's stage
           drain_wait(full_bar(jt % STAGES), (jt / STAGES) & 1u, 50000000ull);
         }
       }
@@ -314,7 +320,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       tc_commit(final_bar);
       drain_wait(final_bar, 0, 100000000ull);
     }
-  } else {
+  } else if (warp < PROD1_WARP) {
     // -------------------------------------------------------- quantizers --
     const int qt = threadIdx.x - 64;
     const int cg = qt & 7;          // group of 16 within the stage's 128 k
@@ -353,7 +359,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       const bool active = kc < c_end;
       // This thread's inputs -> registers: smooth (negated, packed fp32
       // pairs) and x for its one or two rows.
-      uint64_t nsm[8];
+      uint64_t sm2[8];
       uint32_t xv[S::ROWS_PER_THREAD][8];
       uint32_t got = 0;   // depends on every value read from the stage
       if (active) {
@@ -363,11 +369,11 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
           got ^= sa.x ^ sa.y ^ sa.z ^ sa.w ^ sb.x ^ sb.y ^ sb.z ^ sb.w;
           const uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) nsm[j] = bf16x2_to_pk(sw[j] ^ 0x80008000u);
+          for (int j = 0; j < 8; ++j) sm2[j] = bf16x2_to_pk(sw[j]);
         } else {
           // no smoothing: v = x, i.e. a factor of 1 (exact)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) nsm[j] = pk(-1.0f, -1.0f);
+          for (int j = 0; j < 8; ++j) sm2[j] = pk(1.0f, 1.0f);
         }
 #pragma unroll
         for (int rr = 0; rr < S::ROWS_PER_THREAD; ++rr) {
@@ -410,12 +416,12 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       }
       uint32_t sca = 0, scb = 0;
       if (active) {
-        const uint64_t ca = quantize_group(xv[0], nsm, sca);
+        const uint64_t ca = quantize_group(xv[0], sm2, sca);
         if (m0 < p.M)
           *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
               make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
         if constexpr (S::ROWS_PER_THREAD == 2) {
-          const uint64_t cb = quantize_group(xv[S::ROWS_PER_THREAD - 1], nsm, scb);
+          const uint64_t cb = quantize_group(xv[S::ROWS_PER_THREAD - 1], sm2, scb);
           if (m1 < p.M)
             *reinterpret_cast<uint2*>(q1_row + kc * (BKE / 2)) =
                 make_uint2(static_cast<uint32_t>(cb), static_cast<uint32_t>(cb >> 32));
@@ -452,7 +458,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
   // ------------------------------------------------- low-rank readout --
   // TMEM holds L^T: lane r, column m.  The four quantizer warps of lane
   // quarter (warp % 4) read BM / 4 columns each.
-  const bool is_q = warp >= 2;
+  const bool is_q = warp >= 2 && warp < PROD1_WARP;
   const int lq = warp & 3;
   const int slice = (warp - 2) >> 2;
   const int r = lq * 32 + lane;
