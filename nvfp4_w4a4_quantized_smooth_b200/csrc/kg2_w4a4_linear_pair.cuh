@@ -207,9 +207,6 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
-  // Set-up above overlaps the previous kernel; global memory waits for it.
-  griddep_wait();
-  griddep_launch_dependents();
 
   const int num_k = p.K / BK;                  // K steps per tile
   const int uses = num_k + (LR ? 2 : 0);       // stage uses per tile
@@ -221,6 +218,36 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int npairs = static_cast<int>(gridDim.x >> 1);
   const size_t kblocks = static_cast<size_t>(p.K / 64);   // 512-byte scale blocks per 128 rows
+  // The weight side of the first tile's first STAGES stage uses (this CTA's
+  // qweight rows and the tile's weight scales, or its proj_up half) is
+  // requested before the wait for the previous kernel, each use by the
+  // producer that owns it, so that the weight stream overlaps that kernel.
+  const uint32_t pre = pair < tiles ? (uses < STAGES ? static_cast<uint32_t>(uses) : STAGES) : 0u;
+  if ((warp == 0 || warp == PROD1_WARP) && lane == 0) {
+    const uint32_t pid = warp == 0 ? 0u : 1u;
+    const int nb = pair / p.m_tiles;
+    const int brow = nb * BN + static_cast<int>(rank) * BN_CTA;
+    for (uint32_t u = pid; u < pre; u += 2) {
+      const int st = static_cast<int>(u);
+      const uint32_t fb = map_to_rank(full_bar(u), 0);
+      if (!lr_use(st)) {
+        const int ks = st - k0;
+        if (leader) mbar_expect_tx(full_bar(u), 2 * B_BYTES);
+        tma_load_2d_cg2(s_b(u), &tm_b, ks * BK_BYTES, brow, fb);
+        mbar_expect_tx(sfl_bar(u), SFB_BYTES);
+        bulk_load(s_sf(u) + SFA_BYTES,
+                  p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * ks) * 1024, SFB_BYTES,
+                  sfl_bar(u));
+      } else {
+        const int hr = FOLDED ? st : st - num_k;
+        if (leader) mbar_expect_tx(full_bar(u), 2 * LR_B_BYTES);
+        tma_load_2d_cg2(s_b(u), &tm_p, hr * 64, brow, fb);
+      }
+    }
+  }
+  // Set-up above overlaps the previous kernel; what it writes waits for it.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0 || warp == PROD1_WARP) {
     if (lane == 0) {
@@ -253,24 +280,30 @@ w4a4_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [
             break;
           }
           const uint32_t fb = map_to_rank(full_bar(s), 0);
+          const bool weights_in = it < pre;      // weight side requested before the wait
           if (!lr_use(st)) {
             const int ks = st - k0;              // K step
-            if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (A_BYTES + B_BYTES));
+            if (leader)
+              mbar_arrive_expect_tx(full_bar(s), 2 * (A_BYTES + (weights_in ? 0u : B_BYTES)));
             tma_load_2d_cg2(s_a(s), &tm_a, ks * BK_BYTES, arow, fb);
-            tma_load_2d_cg2(s_b(s), &tm_b, ks * BK_BYTES, brow, fb);
-            mbar_arrive_expect_tx(sfl_bar(s), (a_sf ? SFA_BYTES : 0u) + SFB_BYTES);
+            if (!weights_in) tma_load_2d_cg2(s_b(s), &tm_b, ks * BK_BYTES, brow, fb);
+            mbar_arrive_expect_tx(sfl_bar(s),
+                                  (a_sf ? SFA_BYTES : 0u) + (weights_in ? 0u : SFB_BYTES));
             if (a_sf)
               bulk_load(s_sf(s),
                         p.ascales_tiled + (static_cast<size_t>(arow_tile) * kblocks + 4 * ks) * 512,
                         SFA_BYTES, sfl_bar(s));
-            bulk_load(s_sf(s) + SFA_BYTES,
-                      p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * ks) * 1024,
-                      SFB_BYTES, sfl_bar(s));
+            if (!weights_in)
+              bulk_load(s_sf(s) + SFA_BYTES,
+                        p.wscales_tiled + (static_cast<size_t>(nb) * kblocks + 4 * ks) * 1024,
+                        SFB_BYTES, sfl_bar(s));
           } else {
             const int hr = FOLDED ? st : st - num_k;   // which 64-wide half of R
-            if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (LR_A_BYTES + LR_B_BYTES));
+            if (leader)
+              mbar_arrive_expect_tx(full_bar(s),
+                                    2 * (LR_A_BYTES + (weights_in ? 0u : LR_B_BYTES)));
             tma_load_2d_cg2(s_a(s), &tm_l, hr * 64, arow, fb);
-            tma_load_2d_cg2(s_b(s), &tm_p, hr * 64, brow, fb);
+            if (!weights_in) tma_load_2d_cg2(s_b(s), &tm_p, hr * 64, brow, fb);
             // no scales for the low-rank uses; the barrier keeps its phases
             mbar_arrive(sfl_bar(s));
           }

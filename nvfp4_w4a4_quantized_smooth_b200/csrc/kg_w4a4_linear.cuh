@@ -187,13 +187,25 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
-  // Set-up above overlaps the previous kernel; global memory waits for it.
-  griddep_wait();
-  griddep_launch_dependents();
 
   const int num_k = p.K / BK;                  // K steps per tile
   const int tiles = p.m_tiles * p.n_tiles;
   const size_t kblocks = static_cast<size_t>(p.K / 64);   // 512-byte scale blocks per 128 rows
+  // The qweight boxes of the first tile's first AB_SLOTS K steps are
+  // requested before the wait for the previous kernel, so that the weight
+  // stream overlaps it.
+  const int t0 = static_cast<int>(blockIdx.x);
+  const int pre = t0 < tiles ? (num_k < AB_SLOTS ? num_k : AB_SLOTS) : 0;
+  if (warp == 0 && lane == 0) {
+    for (int st = 0; st < pre; ++st) {
+      const uint32_t s = static_cast<uint32_t>(st);
+      mbar_expect_tx(full_bar(s), B_BYTES);
+      tma_load_2d(s_b(s), &tm_b, st * BK_BYTES, (t0 / p.m_tiles) * BN, full_bar(s));
+    }
+  }
+  // Set-up above overlaps the previous kernel; what it writes waits for it.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -211,9 +223,10 @@ w4a4_linear_kernel(const __grid_constant__ CUtensorMap tm_a,   // qact    [M, K/
             break;
           }
           if (st < num_k) {
-            mbar_arrive_expect_tx(full_bar(s), AB_SLOT_BYTES);
+            const bool weights_in = static_cast<int>(it) < pre;   // requested before the wait
+            mbar_arrive_expect_tx(full_bar(s), weights_in ? A_BYTES : AB_SLOT_BYTES);
             tma_load_2d(s_a(s), &tm_a, st * BK_BYTES, mb * BM, full_bar(s));
-            tma_load_2d(s_b(s), &tm_b, st * BK_BYTES, nb * BN, full_bar(s));
+            if (!weights_in) tma_load_2d(s_b(s), &tm_b, st * BK_BYTES, nb * BN, full_bar(s));
           } else {
             const int hr = st - num_k;           // which 64-wide half of R
             mbar_arrive_expect_tx(full_bar(s), LR_A_BYTES + LR_B_BYTES);

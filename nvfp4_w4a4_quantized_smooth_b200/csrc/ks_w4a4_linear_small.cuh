@@ -164,9 +164,6 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot_ptr);
-  // Set-up above overlaps the previous kernel; global memory waits for it.
-  griddep_wait();
-  griddep_launch_dependents();
 
   const int num_k = p.K / BK;                  // K steps per tile
   const int kblocks = p.K / 64;                // 512-byte scale blocks per 128 rows
@@ -178,6 +175,27 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
   const int uses = lr_uses + nk;               // ring slots per tile
   const int tile0 = static_cast<int>(blockIdx.x) / split;
   const int tile_step = static_cast<int>(gridDim.x) / split;
+  // The weight side of the first tile's first SLOTS slots (qweight box and
+  // weight scales, or the proj_up half) is requested before the wait for
+  // the previous kernel, so that the weight stream overlaps it.
+  const int pre = tile0 < p.n_tiles ? (uses < SLOTS ? uses : SLOTS) : 0;
+  if (warp == 0 && lane == 0) {
+    for (int st = 0; st < pre; ++st) {
+      const uint32_t s = static_cast<uint32_t>(st);
+      if (st < lr_uses) {
+        mbar_expect_tx(full_bar(s), LR_A_BYTES);
+        tma_load_2d(s_a(s), &tm_p, st * 64, tile0 * BMW, full_bar(s));
+      } else {
+        const int kk = k0 + st - lr_uses;
+        mbar_expect_tx(full_bar(s), A_BYTES + SFA_BYTES);
+        tma_load_2d(s_a(s), &tm_w, kk * BK_BYTES, tile0 * BMW, full_bar(s));
+        tma_load_3d(s_sf(s), &tm_sw, 0, tile0 & 1, (tile0 >> 1) * kblocks + 4 * kk, full_bar(s));
+      }
+    }
+  }
+  // Set-up above overlaps the previous kernel; what it writes waits for it.
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -192,18 +210,21 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
             ok = false;
             break;
           }
+          const bool weights_in = static_cast<int>(it) < pre;   // requested before the wait
           if (st < lr_uses) {
             const int hr = st;                   // which 64-wide half of R
-            mbar_arrive_expect_tx(full_bar(s), LR_A_BYTES + LR_B_BYTES);
-            tma_load_2d(s_a(s), &tm_p, hr * 64, t * BMW, full_bar(s));
+            mbar_arrive_expect_tx(full_bar(s), (weights_in ? 0u : LR_A_BYTES) + LR_B_BYTES);
+            if (!weights_in) tma_load_2d(s_a(s), &tm_p, hr * 64, t * BMW, full_bar(s));
             tma_load_2d(s_b(s), &tm_l, hr * 64, 0, full_bar(s));
           } else {
             const int kk = k0 + st - lr_uses;    // K step
-            mbar_arrive_expect_tx(full_bar(s), SLOT_BYTES);
-            tma_load_2d(s_a(s), &tm_w, kk * BK_BYTES, t * BMW, full_bar(s));
+            mbar_arrive_expect_tx(full_bar(s), weights_in ? B_BYTES + SFB_BYTES : SLOT_BYTES);
+            if (!weights_in) {
+              tma_load_2d(s_a(s), &tm_w, kk * BK_BYTES, t * BMW, full_bar(s));
+              // weight rows [128 t, 128 t + 128) = half (t & 1) of 256-row tile t / 2
+              tma_load_3d(s_sf(s), &tm_sw, 0, t & 1, (t >> 1) * kblocks + 4 * kk, full_bar(s));
+            }
             tma_load_2d(s_b(s), &tm_x, kk * BK_BYTES, 0, full_bar(s));
-            // weight rows [128 t, 128 t + 128) = half (t & 1) of 256-row tile t / 2
-            tma_load_3d(s_sf(s), &tm_sw, 0, t & 1, (t >> 1) * kblocks + 4 * kk, full_bar(s));
             bulk_load(s_sf(s) + SFA_BYTES, p.ascales_tiled + static_cast<size_t>(4 * kk) * 512,
                       SFB_BYTES, full_bar(s));
           }

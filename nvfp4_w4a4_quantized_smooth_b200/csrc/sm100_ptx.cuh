@@ -52,6 +52,13 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
                : "memory");
 }
 
+// Raise the barrier's expected transaction bytes without an arrival (for
+// copies issued ahead of the arrival that completes the phase's count).
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
                "r"(bytes)
@@ -300,8 +307,11 @@ __device__ __forceinline__ void silu_mul_words(const uint32_t (&a)[NW], const ui
 // A kernel launched with programmatic stream serialization may start while
 // the previous kernel in the stream is still running.  griddep_wait blocks
 // until that kernel has completed and its memory operations are visible;
-// every thread calls it before its first access to global memory.  (No-op
-// for a kernel launched without the attribute.)
+// every thread calls it before it touches memory that kernel may write.
+// The kernels of this library that let their dependents start early (the
+// activation kernel and the GEMMs) never write the weights, so a GEMM may
+// issue the copies of its weight operands before its wait.  (No-op for a
+// kernel launched without the attribute.)
 __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
