@@ -10,11 +10,12 @@
 // its K range (a 128-token x 256-column tile would leave N / 256 CTAs for
 // it).  One CTA per 128 weight rows and K range: with `split` > 1 the K
 // steps of a tile are divided among the `split` CTAs of a thread-block
-// cluster, each of which keeps its fp32 partial tile (and its own copy of
-// the low-rank tile) in shared memory; after a cluster barrier rank r sums
-// the partials of rows [r 128 / split, (r + 1) 128 / split) in rank order
-// through distributed shared memory (deterministic), applies the epilogue
-// and stores those columns of y.  With `split` = 1 a CTA covers the whole
+// cluster: each rank stores the rows of its fp32 partial tile that rank o
+// sums -- rows [o 128 / split, (o + 1) 128 / split) -- into rank o's
+// receive buffer (distributed shared memory stores) and keeps its own copy
+// of the low-rank tile; after one cluster barrier every rank sums its rows
+// over all ranks in rank order from its own shared memory (deterministic),
+// applies the epilogue and stores those columns of y.  With `split` = 1 a CTA covers the whole
 // K range and loops over tiles when there are more than SMs.
 //
 // Roles (192 threads):
@@ -68,8 +69,11 @@ constexpr uint32_t LR_B_BYTES = NT * 64 * 2;         // L half: 64 rows x 64 bf1
 static_assert(LR_A_BYTES <= A_BYTES && LR_B_BYTES <= B_BYTES, "low-rank halves fit a slot");
 constexpr uint32_t RING_BYTES = SLOTS * SLOT_BYTES;
 constexpr uint32_t OUT_BYTES = NT * BMW * 2;         // [64 tokens][128 columns] bf16
+// split > 1: the partial rows every rank sends this one, [rank][token][row]
+// fp32 (split ranks x 64 tokens x 128 / split rows)
+constexpr uint32_t RECV_BYTES = NT * BMW * 4;
 constexpr uint32_t BAR_BYTES = 256;
-constexpr uint32_t SMEM_BYTES = RING_BYTES + OUT_BYTES + BAR_BYTES + 1024;
+constexpr uint32_t SMEM_BYTES = RING_BYTES + OUT_BYTES + RECV_BYTES + BAR_BYTES + 1024;
 constexpr int EPI_WARP0 = 2;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);
@@ -82,6 +86,7 @@ static_assert(TM_SF + SLOTS * TM_SF_SLOT <= TMEM_COLS, "scale columns fit");
 static_assert(SLOT_BYTES % 1024 == 0 && RING_BYTES % 1024 == 0,
               "operand boxes stay 1024-aligned");
 static_assert(8 * 3 * SLOTS + 32 <= BAR_BYTES, "barriers fit");
+static_assert(SMEM_BYTES <= 232448, "fits the shared memory of one SM");
 
 // Wait-site ids recorded in the error word.
 constexpr uint32_t SITE_PROD = 0x40, SITE_MMA_TE = 0x41, SITE_MMA_FULL = 0x42,
@@ -118,12 +123,14 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
   auto s_b = [&](uint32_t s) { return s_ring + s * SLOT_BYTES + A_BYTES; };
   auto s_sf = [&](uint32_t s) { return s_ring + s * SLOT_BYTES + A_BYTES + B_BYTES; };
   const uint32_t s_out = s_ring + RING_BYTES;
-  // After the last MMA (split > 1): this rank's partial and low-rank tiles,
-  // [64 tokens][128 columns] fp32 each, over the first two ring slots.
-  const uint32_t s_part = s_ring;
-  const uint32_t s_lrt = s_ring + NT * BMW * 4;
-  static_assert(2 * NT * BMW * 4 <= RING_BYTES, "partial tiles fit the ring");
-  const uint32_t s_bar = s_out + OUT_BYTES;
+  // After the last MMA (split > 1): this rank's low-rank tile, [64 tokens]
+  // [128 columns] fp32, over the first ring slots (no copy or MMA uses the
+  // ring any more); the receive buffer has its own place, as other ranks
+  // may store into it while this one still runs its K loop.
+  const uint32_t s_lrt = s_ring;
+  static_assert(NT * BMW * 4 <= RING_BYTES, "the low-rank tile fits the ring");
+  const uint32_t s_recv = s_out + OUT_BYTES;
+  const uint32_t s_bar = s_recv + RECV_BYTES;
   // barriers: slot full (TMA bytes), slot scales in TMEM, slot free
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto sf_full_bar = [&](uint32_t s) { return s_bar + 8u * (SLOTS + s); };
@@ -341,10 +348,15 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
       }
       if (ok) ok = __all_sync(0xFFFFFFFFu, svdq_wait(tmem_full_bar, tc & 1u, SITE_EPI));
       if (ok && split > 1) {
-        // This rank's partial tile and its low-rank tile -> shared memory
-        // ([token][column] fp32 at the start of the ring, which no MMA or
-        // copy uses any more), for the cluster sum after the role loops.
+        // This rank's partial rows -> the receive buffer of the rank that
+        // sums them ([rank][token][row - first row of that rank]); its
+        // low-rank tile -> its own shared memory ([token][column] fp32).
         tc_fence_after();
+        const int r0 = BMW / split;
+        const int owner = n_local / r0;
+        const uint32_t recv_o =
+            map_to_rank(s_recv + static_cast<uint32_t>(rank * NT * r0 + (n_local - owner * r0)) * 4u,
+                        static_cast<uint32_t>(owner));
 #pragma unroll
         for (int c = 0; c < NT / 16; ++c) {
           uint32_t acc[16], lr[16];
@@ -358,9 +370,10 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const uint32_t off = static_cast<uint32_t>((16 * c + i) * BMW + n_local) * 4u;
-            st_shared_f32(s_part + off, __uint_as_float(acc[i]));
-            st_shared_f32(s_lrt + off, __uint_as_float(lr[i]));
+            const int m = 16 * c + i;
+            st_dsmem_f32(recv_o + static_cast<uint32_t>(m * r0) * 4u, __uint_as_float(acc[i]));
+            st_shared_f32(s_lrt + static_cast<uint32_t>(m * BMW + n_local) * 4u,
+                          __uint_as_float(lr[i]));
           }
         }
       } else if (ok) {
@@ -406,11 +419,14 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
 
   if (split > 1) {
     // ------------------------------------------------- cluster K sum --
-    // Every thread of every rank takes both cluster barriers.  Rank r sums
-    // rows [r R0, (r + 1) R0) of the partial tiles of all ranks in rank
-    // order; a unit is 4 consecutive rows of one token (a float4 of each
-    // rank's [token][column] tile), so that a warp reads and writes whole
-    // 16-byte pieces.  The low-rank tile is this rank's own copy.
+    // Every thread of every rank takes the cluster barrier, after which
+    // every rank's stores into this rank's receive buffer are visible.
+    // Rank r sums rows [r R0, (r + 1) R0) of all ranks' partial tiles in
+    // rank order; a unit is 4 consecutive rows of one token (a float4 of
+    // each rank's slice), so that a warp reads and writes whole 16-byte
+    // pieces.  The low-rank tile is this rank's own copy.  No rank touches
+    // another's shared memory after the barrier, so none waits for the
+    // others before it exits.
     __syncwarp();
     cluster_sync_all();
     if (warp >= EPI_WARP0 && !error_raised()) {
@@ -423,16 +439,16 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
         const int row = rank * r0 + 4 * (u % groups);
         const int n = t * BMW + row;
         if (m >= p.M || n >= p.N) continue;
-        const uint32_t off = static_cast<uint32_t>(m * BMW + row) * 4u;
-        float4 sum = ld_dsmem_f4(map_to_rank(s_part + off, 0));
+        const uint32_t roff = static_cast<uint32_t>(m * r0 + 4 * (u % groups)) * 4u;
+        float4 sum = ld_shared_f4(s_recv + roff);
         for (int j = 1; j < split; ++j) {
-          const float4 v = ld_dsmem_f4(map_to_rank(s_part + off, j));
+          const float4 v = ld_shared_f4(s_recv + static_cast<uint32_t>(j * NT * r0) * 4u + roff);
           sum.x += v.x;
           sum.y += v.y;
           sum.z += v.z;
           sum.w += v.w;
         }
-        const float4 lr = ld_dsmem_f4(map_to_rank(s_lrt + off, rank));
+        const float4 lr = ld_shared_f4(s_lrt + static_cast<uint32_t>(m * BMW + row) * 4u);
         const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
         const float lv[4] = {lr.x, lr.y, lr.z, lr.w};
         uint32_t packed[2];
@@ -451,8 +467,6 @@ w4a4_linear_small_kernel(const __grid_constant__ CUtensorMap tm_w,   // qweight 
         st_global_v2(p.y + static_cast<size_t>(m) * p.ldy + n, packed[0], packed[1]);
       }
     }
-    __syncwarp();
-    cluster_sync_all();
   }
 
   // ----------------------------------------------------------- teardown --
