@@ -56,10 +56,12 @@
 // rounding as svdq_silu_mul), and the MMA waits for every quantizer warp's
 // part before reading it; x itself is never written to global memory.
 // With split == 1 the tile's L is rounded to bf16 and written directly.
-// Otherwise every rank stages its fp32 partial in its own (idle) stage
-// ring, and after a cluster barrier each rank sums a 1/split slice of the
-// tile over all ranks in rank order (deterministic) through distributed
-// shared memory and writes it as bf16.
+// Otherwise (64-row tiles; split a power of two) rank o sums rows
+// [o BM / split, (o + 1) BM / split) of the tile: every rank stores those
+// rows of its fp32 partial into rank o's receive buffer (distributed
+// shared memory stores), and after one cluster barrier each rank sums its
+// rows over all ranks in rank order (deterministic) from its own shared
+// memory and writes them as bf16.
 #pragma once
 
 #include <cuda.h>
@@ -83,7 +85,6 @@ constexpr int PROD1_WARP = 2 + NUM_QWARPS;   // the second producer
 constexpr int NUM_THREADS = 64 + NUM_QTHREADS + 32;
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM_BUDGET = 227 * 1024;
-constexpr int PART_STRIDE = R + 4;     // floats per row of a staged partial (bank spread)
 constexpr int MAX_SPLIT = 16;
 
 // LR: the layer has the low-rank branch (R = 128); without it (R = 0, the
@@ -98,16 +99,24 @@ struct Shape {
   static constexpr uint32_t X_BYTES = 2 * X_CHUNK;
   static constexpr uint32_t Y_STAGE = SILU ? X_BYTES : 0u;  // the b tile
   static constexpr uint32_t PD_STAGE = LR ? PD_BYTES : 0u;
-  static constexpr uint32_t STAGE_BYTES =
-      (X_BYTES + Y_STAGE + PD_STAGE + SM_BYTES + 1023u) & ~1023u;
-  static constexpr int STAGES_FIT = static_cast<int>((SMEM_BUDGET - BAR_BYTES - 1024) / STAGE_BYTES);
+  // the operand stages (multiples of 1 KB, so every box stays 1024-aligned);
+  // each stage's 256 B of smooth in a small ring of its own after them
+  static constexpr uint32_t STAGE_BYTES = X_BYTES + Y_STAGE + PD_STAGE;
+  // K split (64-row tiles with the low-rank branch): the partial rows the
+  // other ranks send, [rank][row][r] fp32 (split ranks x BM / split rows)
+  static constexpr uint32_t RECV_BYTES = (LR && BM == 64) ? BM * R * 4 : 0u;
+  static constexpr bool CAN_SPLIT = RECV_BYTES > 0;
+  static constexpr int STAGES_FIT = static_cast<int>(
+      (SMEM_BUDGET - BAR_BYTES - 1024 - RECV_BYTES) / (STAGE_BYTES + SM_BYTES));
   static constexpr int MAX_STAGES = LR ? 4 : 8;
   static constexpr int STAGES = STAGES_FIT < MAX_STAGES ? STAGES_FIT : MAX_STAGES;
-  static constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr uint32_t SMEM_BYTES =
+      STAGES * (STAGE_BYTES + SM_BYTES) + RECV_BYTES + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = BM;                 // 64 or 128 (powers of 2)
   static constexpr int ROWS_PER_THREAD = BM / 64;           // 1 or 2
+  static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-aligned");
   static_assert(STAGES >= 3, "at least three stages");
-  static_assert(!LR || BM * PART_STRIDE * 4 <= STAGES * STAGE_BYTES, "partial fits the ring");
+  static_assert(SMEM_BYTES <= SMEM_BUDGET, "fits the shared memory of one SM");
   static_assert(24 * STAGES + 24 <= BAR_BYTES, "barriers fit");
 };
 
@@ -194,15 +203,16 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t s_ring = smem_u32(smem);
-  const uint32_t s_bar = s_ring + STAGES * S::STAGE_BYTES;
-  // Stage layout: x [chunk][BM rows x 128 B], proj_down [r half][128 k x
-  // 128 B], smooth [128 k] bf16.
+  const uint32_t s_smooth = s_ring + STAGES * S::STAGE_BYTES;
+  const uint32_t s_recv = s_smooth + STAGES * SM_BYTES;
+  const uint32_t s_bar = s_recv + S::RECV_BYTES;
+  // Stage layout: x [chunk][BM rows x 128 B], (b [chunk][BM rows x 128 B],)
+  // proj_down [r half][128 k x 128 B]; the stage's smooth [128 k] bf16 in
+  // the smooth ring.
   auto s_x = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES; };
   auto s_y = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES; };
   auto s_pd = [&](uint32_t s) { return s_ring + s * S::STAGE_BYTES + S::X_BYTES + S::Y_STAGE; };
-  auto s_sm = [&](uint32_t s) {
-    return s_ring + s * S::STAGE_BYTES + S::X_BYTES + S::Y_STAGE + S::PD_STAGE;
-  };
+  auto s_sm = [&](uint32_t s) { return s_smooth + s * SM_BYTES; };
   auto full_bar = [&](uint32_t s) { return s_bar + 8u * s; };
   auto empty_bar = [&](uint32_t s) { return s_bar + 8u * (STAGES + s); };
   // SILU: the x slot holds silu(a) * b once every quantizer warp has written
@@ -483,59 +493,49 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
         if (m < p.M) p.lowrank[static_cast<size_t>(m) * R + r] = __float2bfloat16_rn(__uint_as_float(v[j]));
       }
     }
-  } else {
-    // Partial sums: every quantizer warp has finished with the ring (and
-    // every MMA has completed) before any of them overwrites it with its
-    // fp32 partial (row-major [m][r], PART_STRIDE floats per row).
-    if (is_q) {
-      named_bar_sync(1, NUM_QTHREADS);
-      if (l_ready) {
-        tc_fence_after();
-        uint32_t v[CW];
-        if constexpr (CW == 32) {
-          tmem_ld_32x32b_x32(lane_addr, v);
-        } else {
-          tmem_ld_32x32b_x16(lane_addr, v);
-        }
-        tmem_ld_wait();
+  } else if constexpr (S::CAN_SPLIT) {
+    // Rank o sums rows [o RO, (o + 1) RO) of the tile (RO = BM / split):
+    // every rank stores those rows of its fp32 partial into rank o's
+    // receive buffer ([rank][row - o RO][r]); rank o's buffer is used for
+    // nothing else, so the stores may land while o still runs its K loop.
+    const int ro = BM / p.split;
+    if (is_q && l_ready) {
+      tc_fence_after();
+      uint32_t v[CW];
+      if constexpr (CW == 32) {
+        tmem_ld_32x32b_x32(lane_addr, v);
+      } else {
+        tmem_ld_32x32b_x16(lane_addr, v);
+      }
+      tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < CW; ++j)
-          asm volatile("st.shared.f32 [%0], %1;" ::"r"(s_ring + ((mc + j) * PART_STRIDE + r) * 4),
-                       "f"(__uint_as_float(v[j]))
-                       : "memory");
+      for (int j = 0; j < CW; ++j) {
+        const int m = mc + j;
+        const int o = m / ro;
+        const uint32_t idx = static_cast<uint32_t>((rank * ro + (m - o * ro)) * R + r);
+        st_dsmem_f32(map_to_rank(s_recv + 4u * idx, static_cast<uint32_t>(o)), __uint_as_float(v[j]));
       }
     }
+    // After the barrier every rank's stores into this rank's buffer are
+    // visible; no rank touches another's shared memory after it, so none
+    // waits for the others before it exits.
     __syncwarp();
     cluster_sync_all();
     if (is_q && !error_raised()) {
-      // This rank sums its share of the BM x 32 float4 units over all ranks.
-      const int units = BM * (R / 4);
-      const int u0 = rank * units / p.split;
-      const int u1 = (rank + 1) * units / p.split;
-      for (int u = u0 + (threadIdx.x - 64); u < u1; u += NUM_QTHREADS) {
-        const int m = u / (R / 4);
+      // A unit is 4 consecutive r of one row: the float4 of each rank's
+      // slice, summed in rank order.
+      for (int u = threadIdx.x - 64; u < ro * (R / 4); u += NUM_QTHREADS) {
+        const int mr = u / (R / 4);
         const int c4 = u % (R / 4);
-        const uint32_t off = s_ring + (m * PART_STRIDE + 4 * c4) * 4;
-        // Eight ranks' values are requested before their first add (the
-        // remote loads overlap); the sum still runs in rank order.
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int b0 = 0; b0 < p.split; b0 += 8) {
-          float4 t[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (b0 + j < p.split)
-              t[j] = ld_dsmem_f4(map_to_rank(off, static_cast<uint32_t>(b0 + j)));
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (b0 + j < p.split) {
-              acc.x += t[j].x;
-              acc.y += t[j].y;
-              acc.z += t[j].z;
-              acc.w += t[j].w;
-            }
-          }
+        for (int b = 0; b < p.split; ++b) {
+          const float4 t = ld_shared_f4(s_recv + 4u * static_cast<uint32_t>((b * ro + mr) * R + 4 * c4));
+          acc.x += t.x;
+          acc.y += t.y;
+          acc.z += t.z;
+          acc.w += t.w;
         }
-        const int row = mb * BM + m;
+        const int row = mb * BM + rank * ro + mr;
         if (row < p.M) {
           __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
           __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
@@ -544,9 +544,6 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
         }
       }
     }
-    // No rank leaves while another may still read its shared memory.
-    __syncwarp();
-    cluster_sync_all();
   }
 
   // ----------------------------------------------------------- teardown --

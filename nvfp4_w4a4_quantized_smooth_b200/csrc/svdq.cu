@@ -458,7 +458,9 @@ int kq_max_clusters(DeviceInfo* d, int bm, int split) {
 // among the grids that run in one wave (at most one CTA per SM, every
 // cluster co-resident), the one that occupies the most SMs; ties go to the
 // tile height that pads M the least, then to the taller tile (less
-// proj_down traffic per row), then to the smaller split.
+// proj_down traffic per row), then to the smaller split.  A split takes
+// 64-row tiles (the kernel's receive buffer for the partial sums fits
+// beside four stages only there).
 // If none fits (very large M), 128-row tiles without a split.
 // A K split gives every CTA at least 256 k (4 chunks of 64) up to 8 ranks,
 // and at least one 128-k stage with 16 ranks (a non-portable cluster size,
@@ -478,6 +480,7 @@ void kq_plan(DeviceInfo* d, int M, int K, int* bm_out, int* split_out, bool tall
          split *= 2) {
       const int ctas = m_tiles * split;
       if (ctas > d->num_sms) break;
+      if (split > 1 && bm != 64) continue;
       if (split > 1 && m_tiles > kq_max_clusters(d, bm, split)) continue;
       if (ctas > best_ctas || (ctas == best_ctas && pad < best_pad)) {
         best_ctas = ctas;
@@ -629,6 +632,7 @@ int quantize_act_impl(const uint16_t* a, const uint16_t* b, int M, int K, int ld
     kq_plan(d, M, K, &bm, &split, /*tall_ok=*/!silu);
   else
     kq_plan_plain(d, M, K, &bm, &split);
+  if (lr && split > 1 && bm != 64) return SVDQ_ERR_UNSUPPORTED;   // the plan never does this
   const int m_tiles = (M + bm - 1) / bm;
 
   // x (a, b) viewed as {64 k, M rows, K/64 chunks} and proj_down as {64 r,

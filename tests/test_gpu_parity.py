@@ -85,6 +85,7 @@ def test_quantize_plans_fit_one_wave():
             tiles = -(-M // bm)
             assert bm in (64, 128), (M, K, bm)
             assert split in (1, 2, 4, 8, 16), (M, K, split)
+            assert split == 1 or bm == 64, (M, K, bm, split)   # a split takes 64-row tiles
             assert split == 1 or (256 if split <= 8 else 128) * split <= K, (M, K, split)
             if tiles * split > sms:
                 assert split == 1 and bm == 128, (M, K, bm, split)
