@@ -288,10 +288,11 @@ int svdq_quantize_weights_noalloc(const uint16_t* W, const uint16_t* smooth, con
 /* ---- helpers ------------------------------------------------------------ */
 
 /* Launch shape svdq_quantize_act uses on the current device for an [M, K]
- * input with the low-rank branch (R = 128): rows per tile (*bm, 64 or 128) and the number of K ranges per
- * tile (*split: 1, 2, 4, 8 or 16 CTAs of a cluster, at least 256 k each
- * up to 8 and at least 128 k each with 16),
- * chosen to occupy the most SMs in one wave.  The K ranges of a tile are
+ * input with the low-rank branch (R = 128): rows per tile (*bm, 64 or 128)
+ * and the number of K ranges per tile (*split: 1, 2, 4, 8 or 16 CTAs of a
+ * cluster, at least 256 k each up to 8 and at least 128 k each with 16; a
+ * split always takes 64-row tiles), chosen to occupy the most SMs in one
+ * wave.  The K ranges of a tile are
  * [r * (K/64) / split, (r + 1) * (K/64) / split) in units of 64 k, so they
  * differ by at most 64 k when K/64 is not a multiple of split.  The
  * summation order of L (and so its last bits) depends on this plan, which
