@@ -26,7 +26,10 @@
 // bits) and an exact midpoint comes out exactly.  Both parts are >= 0, so
 // the sign of a zero v is kept (v r_lo and v r_hi carry it, and zeros of
 // one sign add to that sign); a scale that rounds to zero gives r_hi =
-// r_lo = 0 and therefore signed zero codes.
+// r_lo = 0 and therefore signed zero codes.  With the low-rank branch r_hi
+// comes from a table of the 128 scale codes, filled once per CTA with the
+// same __frcp_rd (the same values; the other instances' rings fill the
+// shared memory, so they compute it per group).
 
 // CTA work item: a tile of BM rows (64 or 128, a template parameter) and
 // one of `split` ranges of K; the `split` CTAs of a tile form a
@@ -106,12 +109,16 @@ struct Shape {
   // other ranks send, [rank][row][r] fp32 (split ranks x BM / split rows)
   static constexpr uint32_t RECV_BYTES = (LR && BM == 64) ? BM * R * 4 : 0u;
   static constexpr bool CAN_SPLIT = RECV_BYTES > 0;
+  // with the low-rank branch: 1/d rounded down for each of the 128 scale
+  // codes (the other instances compute it per group: their rings fill the
+  // shared memory)
+  static constexpr uint32_t RCP_BYTES = LR ? 512u : 0u;
   static constexpr int STAGES_FIT = static_cast<int>(
-      (SMEM_BUDGET - BAR_BYTES - 1024 - RECV_BYTES) / (STAGE_BYTES + SM_BYTES));
+      (SMEM_BUDGET - BAR_BYTES - 1024 - RECV_BYTES - RCP_BYTES) / (STAGE_BYTES + SM_BYTES));
   static constexpr int MAX_STAGES = LR ? 4 : 8;
   static constexpr int STAGES = STAGES_FIT < MAX_STAGES ? STAGES_FIT : MAX_STAGES;
   static constexpr uint32_t SMEM_BYTES =
-      STAGES * (STAGE_BYTES + SM_BYTES) + RECV_BYTES + BAR_BYTES + 1024;
+      STAGES * (STAGE_BYTES + SM_BYTES) + RECV_BYTES + RCP_BYTES + BAR_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = BM;                 // 64 or 128 (powers of 2)
   static constexpr int ROWS_PER_THREAD = BM / 64;           // 1 or 2
   static_assert(STAGE_BYTES % 1024 == 0, "stages stay 1024-aligned");
@@ -156,7 +163,8 @@ __device__ __forceinline__ uint64_t bf16x2_to_pk(uint32_t w) {
 // scale byte.
 __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
                                                    const uint64_t (&sm2)[8],
-                                                   uint32_t& scale_byte) {
+                                                   uint32_t& scale_byte,
+                                                   const float* __restrict__ rhi_tab = nullptr) {
   uint64_t v[8];
   float m8[8];
 #pragma unroll
@@ -174,7 +182,10 @@ __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
   scale_byte = sc;
   const float d = e4m3_to_f32(sc);
   float r_hi = 0.0f, r_lo = 0.0f;
-  if (d > 0.0f) {
+  if (rhi_tab != nullptr) {
+    r_hi = rhi_tab[sc];                      // 0 for a zero scale
+    r_lo = fmaf(-d, r_hi, 1.0f) * r_hi;
+  } else if (d > 0.0f) {
     r_hi = __frcp_rd(d);
     r_lo = fmaf(-d, r_hi, 1.0f) * r_hi;
   }
@@ -200,12 +211,14 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
   using S = Shape<BM, LR, SILU>;
   constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-aligned, derived from the shared array so that plain accesses
+  // through it stay shared-memory accesses
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t s_ring = smem_u32(smem);
   const uint32_t s_smooth = s_ring + STAGES * S::STAGE_BYTES;
   const uint32_t s_recv = s_smooth + STAGES * SM_BYTES;
-  const uint32_t s_bar = s_recv + S::RECV_BYTES;
+  const uint32_t s_rcp = s_recv + S::RECV_BYTES;
+  const uint32_t s_bar = s_rcp + S::RCP_BYTES;
   // Stage layout: x [chunk][BM rows x 128 B], (b [chunk][BM rows x 128 B],)
   // proj_down [r half][128 k x 128 B]; the stage's smooth [128 k] bf16 in
   // the smooth ring.
@@ -355,6 +368,18 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
                    (m1 & 31) * 16 + ((m1 & 127) >> 5) * 4;
     // rows the tiled scale buffer holds (M rounded up to 128)
     const int rows_pad = (p.M + 127) & ~127;
+    // The table of 1/d rounded down, filled once by the first 128
+    // quantizer threads with the same operation as the per-group path.
+    const float* rhi_tab = nullptr;
+    if constexpr (LR) {
+      float* tab = reinterpret_cast<float*>(smem + (s_rcp - s_ring));
+      if (qt < 128) {
+        const float d = e4m3_to_f32(static_cast<uint32_t>(qt));
+        tab[qt] = d > 0.0f ? __frcp_rd(d) : 0.0f;
+      }
+      named_bar_sync(1, NUM_QTHREADS);
+      rhi_tab = tab;
+    }
     bool ok = true;
     for (int i = 0; i < nstages; ++i) {
       const uint32_t s = static_cast<uint32_t>(i) % STAGES;
@@ -374,8 +399,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       uint32_t got = 0;   // depends on every value read from the stage
       if (active) {
         if (p.smooth != nullptr) {
-          const uint4 sa = lds_v4(s_sm(s) + cg * 32);
-          const uint4 sb = lds_v4(s_sm(s) + cg * 32 + 16);
+          const uint4 sa = *reinterpret_cast<const uint4*>(smem + (s_sm(s) - s_ring) + cg * 32);
+          const uint4 sb =
+              *reinterpret_cast<const uint4*>(smem + (s_sm(s) - s_ring) + cg * 32 + 16);
           got ^= sa.x ^ sa.y ^ sa.z ^ sa.w ^ sb.x ^ sb.y ^ sb.z ^ sb.w;
           const uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
 #pragma unroll
@@ -390,7 +416,7 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const uint32_t off = (hh ? xo1 : xo0) + rr * 64 * 128;
-            uint4 v4 = lds_v4(s_x(s) + off);
+            uint4 v4 = *reinterpret_cast<const uint4*>(smem + (s_x(s) - s_ring) + off);
             got ^= v4.x ^ v4.y ^ v4.z ^ v4.w;
             if constexpr (SILU) {
               // x = silu(a) * b, written over a in the x slot (same
@@ -426,29 +452,24 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       }
       uint32_t sca = 0, scb = 0;
       if (active) {
-        const uint64_t ca = quantize_group(xv[0], sm2, sca);
+        const uint64_t ca = quantize_group(xv[0], sm2, sca, rhi_tab);
         if (m0 < p.M)
           *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
               make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
         if constexpr (S::ROWS_PER_THREAD == 2) {
-          const uint64_t cb = quantize_group(xv[S::ROWS_PER_THREAD - 1], sm2, scb);
+          const uint64_t cb = quantize_group(xv[S::ROWS_PER_THREAD - 1], sm2, scb, rhi_tab);
           if (m1 < p.M)
             *reinterpret_cast<uint2*>(q1_row + kc * (BKE / 2)) =
                 make_uint2(static_cast<uint32_t>(cb), static_cast<uint32_t>(cb >> 32));
         }
       }
-      // Lanes 4j..4j+3 hold one row's four groups of one chunk.
-      uint32_t wa = sca << (8 * g);
-      wa |= __shfl_xor_sync(0xFFFFFFFFu, wa, 1);
-      wa |= __shfl_xor_sync(0xFFFFFFFFu, wa, 2);
-      if (active && g == 0 && m0 < rows_pad)
-        *reinterpret_cast<uint32_t*>(sc0 + static_cast<size_t>(kc) * 512) = wa;
+      // Each thread stores its group's scale byte (byte g of the row's
+      // word for the chunk).
+      if (active && m0 < rows_pad)
+        sc0[static_cast<size_t>(kc) * 512 + g] = static_cast<uint8_t>(sca);
       if constexpr (S::ROWS_PER_THREAD == 2) {
-        uint32_t wb = scb << (8 * g);
-        wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 1);
-        wb |= __shfl_xor_sync(0xFFFFFFFFu, wb, 2);
-        if (active && g == 0 && m1 < rows_pad)
-          *reinterpret_cast<uint32_t*>(sc1 + static_cast<size_t>(kc) * 512) = wb;
+        if (active && m1 < rows_pad)
+          sc1[static_cast<size_t>(kc) * 512 + g] = static_cast<uint8_t>(scb);
       } else {
         // 64-row tiles may end half way through the last 128-row scale
         // block: the last tile also writes the zero scales of the rows
