@@ -147,29 +147,34 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ float rcp_approx(float x) {
-  float r;
-  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
+// x * smooth for one word of each (two bf16 values, element 2i in the low
+// half) -> packed fp32 pair: a bf16 x bf16 product is exact in fp32, and
+// the mixed-precision FMA forms it straight from the 16-bit halves; the
+// addend -0 keeps the product's sign when it is zero (+0 + -0 = +0,
+// -0 + -0 = -0).
+__device__ __forceinline__ uint64_t mul_bf16x2(uint32_t x, uint32_t s) {
+  float lo, hi;
+  asm("{\n\t.reg .b16 xl, xh, sl, sh;\n\t"
+      "mov.b32 {xl, xh}, %2;\n\t"
+      "mov.b32 {sl, sh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, xl, sl, 0f80000000;\n\t"
+      "fma.rn.f32.bf16 %1, xh, sh, 0f80000000;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(x), "r"(s));
+  return pk(lo, hi);
 }
 
-// bf16 pair word -> packed fp32 pair (element 2i in the low word).
-__device__ __forceinline__ uint64_t bf16x2_to_pk(uint32_t w) {
-  return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-
-// One 16-element group: x (8 bf16x2 words) and the smooth values as packed
-// fp32 pairs -> 16 E2M1 codes (element 0 in the lowest nibble) and the e4m3
-// scale byte.
+// One 16-element group: x and the smooth values (8 bf16x2 words each) ->
+// 16 E2M1 codes (element 0 in the lowest nibble) and the e4m3 scale byte.
 __device__ __forceinline__ uint64_t quantize_group(const uint32_t (&xw)[8],
-                                                   const uint64_t (&sm2)[8],
+                                                   const uint32_t (&sw)[8],
                                                    uint32_t& scale_byte,
                                                    const float* __restrict__ rhi_tab = nullptr) {
   uint64_t v[8];
   float m8[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    v[i] = mul2(bf16x2_to_pk(xw[i]), sm2[i]);
+    v[i] = mul_bf16x2(xw[i], sw[i]);
     float lo, hi;
     upk(v[i], lo, hi);
     m8[i] = fmaxf(fabsf(lo), fabsf(hi));
@@ -392,9 +397,9 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       // In a range's last stage the second chunk may be absent: those lanes
       // compute nothing but still take part in the shuffles below.
       const bool active = kc < c_end;
-      // This thread's inputs -> registers: smooth (negated, packed fp32
-      // pairs) and x for its one or two rows.
-      uint64_t sm2[8];
+      // This thread's inputs -> registers: smooth and x for its one or two
+      // rows (bf16 pairs).
+      uint32_t sw[8];
       uint32_t xv[S::ROWS_PER_THREAD][8];
       uint32_t got = 0;   // depends on every value read from the stage
       if (active) {
@@ -403,13 +408,12 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
           const uint4 sb =
               *reinterpret_cast<const uint4*>(smem + (s_sm(s) - s_ring) + cg * 32 + 16);
           got ^= sa.x ^ sa.y ^ sa.z ^ sa.w ^ sb.x ^ sb.y ^ sb.z ^ sb.w;
-          const uint32_t sw[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) sm2[j] = bf16x2_to_pk(sw[j]);
+          sw[0] = sa.x; sw[1] = sa.y; sw[2] = sa.z; sw[3] = sa.w;
+          sw[4] = sb.x; sw[5] = sb.y; sw[6] = sb.z; sw[7] = sb.w;
         } else {
           // no smoothing: v = x, i.e. a factor of 1 (exact)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) sm2[j] = pk(1.0f, 1.0f);
+          for (int j = 0; j < 8; ++j) sw[j] = 0x3F803F80u;
         }
 #pragma unroll
         for (int rr = 0; rr < S::ROWS_PER_THREAD; ++rr) {
@@ -452,12 +456,12 @@ quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,    // x (or a) {64
       }
       uint32_t sca = 0, scb = 0;
       if (active) {
-        const uint64_t ca = quantize_group(xv[0], sm2, sca, rhi_tab);
+        const uint64_t ca = quantize_group(xv[0], sw, sca, rhi_tab);
         if (m0 < p.M)
           *reinterpret_cast<uint2*>(q0_row + kc * (BKE / 2)) =
               make_uint2(static_cast<uint32_t>(ca), static_cast<uint32_t>(ca >> 32));
         if constexpr (S::ROWS_PER_THREAD == 2) {
-          const uint64_t cb = quantize_group(xv[S::ROWS_PER_THREAD - 1], sm2, scb, rhi_tab);
+          const uint64_t cb = quantize_group(xv[S::ROWS_PER_THREAD - 1], sw, scb, rhi_tab);
           if (m1 < p.M)
             *reinterpret_cast<uint2*>(q1_row + kc * (BKE / 2)) =
                 make_uint2(static_cast<uint32_t>(cb), static_cast<uint32_t>(cb >> 32));
