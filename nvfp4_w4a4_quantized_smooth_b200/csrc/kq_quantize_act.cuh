@@ -6,7 +6,8 @@
 // Quantization of each 16-element group along K (one e4m3 scale per 16 k,
 // E2M1 elements, as the card's first paragraph states; rounding to
 // nearest-even with saturation):
-//   v = x * smooth                  exact in fp32 (bf16 x bf16)
+//   v = x * smooth                  exact in fp32 (bf16 x bf16, formed by
+//                                   the mixed-precision FMA)
 //   s = e4m3(amax|v| / 6)           quotient, then the hardware RNE /
 //                                   satfinite conversion
 //   q = E2M1(v / s)                 quotient, then the hardware RNE /
@@ -46,9 +47,9 @@
 //               accumulator in BM TMEM columns.
 //   warps 2..17 quantizers: thread t owns 16-element group (t % 8) of the
 //               stage's 128 k and row t / 8 (and t / 8 + 64 when BM = 128,
-//               two independent groups side by side); it converts its 16
-//               smooth values once per stage; writes packed codes and tiled
-//               scales; afterwards reads L^T out of TMEM.
+//               two independent groups side by side); it reads its 16
+//               smooth values once per stage; writes packed codes and its
+//               scale bytes; afterwards reads L^T out of TMEM.
 // Without the low-rank branch (R = 0, the plain NVFP4 layer; template
 // parameter LR = false) the same kernel only quantizes: no proj_down, MMA,
 // TMEM or cluster, and a deeper ring of x stages.  A null smooth means no
